@@ -1,0 +1,532 @@
+#!/usr/bin/env python
+"""Throughput of the MoE dispatch/combine hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole path over one batch of the 4096-token
+prefill workload (hidden 7168, 256 experts in 8 logical ranks, top-8,
+group-limited routing): dispatch layout, bf16 dispatch, FP8 dispatch, and
+the gate-weighted combine of the bf16 receive buffer (identity experts).
+Inputs are resident in HBM when the timed region starts; L2 is flushed
+(256 MiB write) between steps, outside the per-step CUDA events.
+
+Prints one JSON line.  ``value`` is algorithmic HBM bytes moved per second
+over all ranks (each source byte read once, each destination byte written
+once); ``roofline`` is the dominant kernel against the measured copy
+bandwidth; ``decode`` is the 128-token decode workload in microseconds per
+call (layout + FP8 dispatch + combine), plain and in a CUDA graph;
+``cpu_baseline`` times the CPU oracle on a bounded sample; ``e2e`` runs the
+same step from pinned host buffers with the copies inside the timed region.
+
+Under torchrun (N > 1) every rank runs its own batch (weak scaling, no
+data-path collective); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = ("dispatch+combine HBM GB/s (% of B200 peak); "
+          "µs/call at 128-token decode")
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------- bytes model
+
+def step_bytes(T: int, H: int, k: int, E: int, R: int) -> dict:
+    """Algorithmic bytes per kernel of one step: each source byte read once,
+    each destination byte written once (index arrays counted for layout
+    only)."""
+    N = T * k
+    layout = T * k * 8 + (2 * E + 1 + 2 * R + 1) * 4 + T * R + 2 * N * 4
+    return {
+        "layout": layout,
+        "dispatch_bf16": T * H * 2 + N * H * 2,
+        "dispatch_fp8": T * H * 2 + N * H + N * (H // 128) * 4,
+        "combine": N * H * 2 + T * H * 2,
+    }
+
+
+def decode_bytes(T, H, k, E, R) -> int:
+    b = step_bytes(T, H, k, E, R)
+    return b["layout"] + b["dispatch_fp8"] + b["combine"]
+
+
+# --------------------------------------------------------------- utilities
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        # address the GPU by UUID: local CUDA indices may be remapped
+        try:
+            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:  # noqa: BLE001 - older torch without .uuid
+            self.dev = str(device.index)
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "200"], stdout=self.file,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return None
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------- the timed path
+
+class Step:
+    """Device buffers and the calls of one step on one GPU."""
+
+    def __init__(self, ep, cfg, batch, device):
+        self.ep, self.cfg, self.dev = ep, cfg, device
+        T, H, k, E, R = batch.T, batch.H, cfg.k, cfg.E, cfg.R
+        self.T, self.H = T, H
+        self.idx = batch.idx.to(device)
+        self.x = batch.x.to(device)
+        self.w = batch.w.to(device)
+        self.layout = ep.empty_layout(T, k, E, R, device)
+        nws = ep.ep_layout_workspace_bytes(T, k, E, R)
+        self.ws = torch.zeros(max(nws, 16), dtype=torch.uint8, device=device)
+        self.d_err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.recv = torch.empty((T * k, H), dtype=torch.bfloat16, device=device)
+        self.recv_q = torch.empty((T * k, H), dtype=torch.float8_e4m3fn, device=device)
+        self.recv_s = torch.empty((T * k, H // 128), dtype=torch.float32, device=device)
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+
+    def run(self, stream, events=None, fp8_only=False):
+        ep, c = self.ep, self.cfg
+        if events is not None:
+            events[0].record(stream)
+        ep.ep_get_layout(self.idx, c.E, c.R, out=self.layout, ws=self.ws,
+                         d_err=self.d_err, stream=stream)
+        if events is not None:
+            events[1].record(stream)
+        if not fp8_only:
+            ep.ep_dispatch(self.x, self.layout.slot_pos, recv=self.recv, stream=stream)
+        if events is not None:
+            events[2].record(stream)
+        ep.ep_dispatch(self.x, self.layout.slot_pos, fp8=True, recv=self.recv_q,
+                       recv_scale=self.recv_s, stream=stream)
+        if events is not None:
+            events[3].record(stream)
+        ep.ep_combine(self.recv, self.layout.slot_pos, self.w, out=self.out, stream=stream)
+        if events is not None:
+            events[4].record(stream)
+
+
+KERNELS = ("layout", "dispatch_bf16", "dispatch_fp8", "combine")
+
+
+def bench_ours(args, world, rank, device):
+    import combine_ep_get_09_b200 as ep
+    ep.lib()
+    cfg = workloads.CONFIGS["prefill"]
+    batch = workloads.make_batch(cfg, seed=rank)
+    st = Step(ep, cfg, batch, device)
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    nbytes = step_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R)
+    total_bytes = sum(nbytes.values())
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            st.run(stream)
+    stream.synchronize()
+    if ep.ep_read_error(st.d_err, stream) != 0:
+        raise RuntimeError("device reported a bad expert id")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(device)
+    launches0 = ep.ep_kernel_launches()
+    with ClockSampler(device) as clocks, torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            st.run(stream, evs[i])
+        stream.synchronize()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    launches = ep.ep_kernel_launches() - launches0
+
+    per_kernel = {n: [] for n in KERNELS}
+    step_ms = []
+    for e in evs:
+        for j, n in enumerate(KERNELS):
+            per_kernel[n].append(e[j].elapsed_time(e[j + 1]))
+        step_ms.append(e[0].elapsed_time(e[4]))
+    total_ms = max_over_ranks(sum(step_ms), world, device)
+    kern_ms = {n: max_over_ranks(statistics.mean(v), world, device) for n, v in per_kernel.items()}
+
+    peak, peak_kind = measured_peak()
+    kernels = {}
+    for n in KERNELS:
+        gbs = nbytes[n] / (kern_ms[n] * 1e-3) / 1e9
+        kernels[n] = {"us": round(kern_ms[n] * 1e3, 2), "bytes": nbytes[n],
+                      "GB/s": round(gbs, 1), "frac_of_measured": round(gbs / peak, 4),
+                      "frac_of_8TBs": round(gbs / SPEC_HBM_GBS, 4)}
+    dom = max(("dispatch_bf16", "dispatch_fp8", "combine"), key=lambda n: kern_ms[n])
+    dom_gbs = nbytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
+    traffic = profiled_traffic(dom)
+
+    value = world * total_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": ("prefill: T=4096 tokens, H=7168, E=256 experts in R=8 "
+                         "logical ranks, top-8 group-limited routing; step = "
+                         "layout + bf16 dispatch + FP8 dispatch + combine"),
+            "T": cfg.T, "H": cfg.H, "E": cfg.E, "R": cfg.R, "k": cfg.k,
+            "bytes_per_step": total_bytes,
+            "l2": "flushed between steps (256 MiB write), outside the step events",
+            "parallelism": f"{world} independent batch(es), one per GPU",
+        },
+        "frac_of_8TBs": round(value / world / SPEC_HBM_GBS, 4),
+        "kernels": kernels,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(dom_gbs / peak, 4),
+                     "traffic": traffic,
+                     "algorithmic_bytes": nbytes[dom]},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if not args.skip_decode:
+        result["decode"] = bench_decode(ep, device, world)
+    if not args.skip_e2e:
+        result["e2e"] = bench_e2e(ep, cfg, batch, device, args, world, total_bytes)
+    if world == 1 and rank == 0 and not args.skip_cpu:
+        result["cpu_baseline"] = cpu_baseline(cfg, batch, args.cpu_seconds)
+    return result
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary of `kernel`,
+    valid only while the library sources are the ones profiled."""
+    from combine_ep_get_09_b200 import build as lib_build
+    path = os.path.join(ROOT, "profiles", f"{kernel}_prefill.md")
+    try:
+        with open(path) as f:
+            text = f.read()
+    except OSError:
+        return None
+    m = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m or not t or m.group(1) != lib_build.source_digest():
+        return None
+    return float(t.group(1))
+
+
+def bench_decode(ep, device, world, iters=200):
+    cfg = workloads.CONFIGS["decode"]
+    batch = workloads.make_batch(cfg, seed=100)
+    st = Step(ep, cfg, batch, device)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for _ in range(20):
+            st.run(stream, fp8_only=True)
+    stream.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(iters):
+            st.run(stream, fp8_only=True)
+        b.record(stream)
+    stream.synchronize()
+    us_stream = a.elapsed_time(b) * 1e3 / iters
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        st.run(stream, fp8_only=True)
+    with torch.cuda.stream(stream):
+        for _ in range(20):
+            g.replay()
+        a.record(stream)
+        for _ in range(iters):
+            g.replay()
+        b.record(stream)
+    stream.synchronize()
+    us_graph = a.elapsed_time(b) * 1e3 / iters
+    del g
+    us_stream = max_over_ranks(us_stream, world, device)
+    us_graph = max_over_ranks(us_graph, world, device)
+    nb = decode_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R)
+    return {"workload": "decode: T=128, H=7168, E=256/R=8, top-8, FP8 dispatch; "
+                        "call = layout + FP8 dispatch + combine",
+            "us_per_call_graph": round(us_graph, 2),
+            "us_per_call_stream": round(us_stream, 2),
+            "bytes_per_call": nb,
+            "GB/s_graph": round(nb / (us_graph * 1e-6) / 1e9, 1),
+            "l2": "warm (back-to-back calls; the working set fits in L2)",
+            "pages_context_us": 163.0}
+
+
+def bench_e2e(ep, cfg, batch, device, args, world, total_bytes):
+    """Same step from pinned host buffers: H2D of idx, w, x, the four calls,
+    D2H of the combined output, all inside the events."""
+    T, H, k = cfg.T, cfg.H, cfg.k
+    h_idx = batch.idx.pin_memory()
+    h_w = batch.w.pin_memory()
+    h_x = batch.x.pin_memory()
+    h_out = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    st = Step(ep, cfg, batch, device)
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def one(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        st.idx.copy_(h_idx, non_blocking=True)
+        st.w.copy_(h_w, non_blocking=True)
+        st.x.copy_(h_x, non_blocking=True)
+        st.run(stream)
+        h_out.copy_(st.out, non_blocking=True)
+        if evs is not None:
+            evs[1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            one()
+    stream.synchronize()
+    n = max(3, min(args.steps, 10))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    barrier(world)
+    with torch.cuda.stream(stream):
+        for i in range(n):
+            flush.zero_()
+            one(evs[i])
+    stream.synchronize()
+    barrier(world)
+    ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), world, device)
+    h2d = h_idx.numel() * 8 + h_w.numel() * 4 + h_x.numel() * 2
+    d2h = h_out.numel() * 2
+    return {"value": round(world * total_bytes * n / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / n, 4), "steps": n}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_sample_step(oracle, cfg, x, idx, w):
+    """One pass of the oracle over a token sample: layout, bf16 dispatch,
+    FP8 dispatch, combine (identity experts)."""
+    T, k = idx.shape
+    L = oracle.layout(idx, cfg.E, cfg.R)
+    recv = oracle.dispatch_bf16(x, L["slot_pos"], T * k)
+    oracle.dispatch_fp8(x, L["slot_pos"], T * k)
+    oracle.combine(recv, L["slot_pos"], w)
+
+
+def cpu_baseline(cfg, batch, seconds: float, sample_tokens: int = 512):
+    import oracle
+    x = batch.x[:sample_tokens].contiguous()
+    idx = batch.idx[:sample_tokens].contiguous()
+    w = batch.w[:sample_tokens].contiguous()
+    nb = sum(step_bytes(sample_tokens, cfg.H, cfg.k, cfg.E, cfg.R).values())
+    oracle_sample_step(oracle, cfg, x, idx, w)        # warm
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_sample_step(oracle, cfg, x, idx, w)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": round(nb * reps / el / 1e9, 3), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": (f"first {sample_tokens} tokens of the prefill batch, whole step "
+                       f"(layout + bf16 dispatch + FP8 dispatch + combine), "
+                       f"{reps} reps in {el:.1f} s, single-threaded C oracle")}
+
+
+def bench_reference(args, world, rank):
+    """The oracle as it stands, timed on the host cores: same metric, unit
+    and workload, each step a bounded token sample of the prefill batch."""
+    if rank != 0:
+        return None
+    import oracle
+    cfg = workloads.CONFIGS["prefill"]
+    batch = workloads.make_batch(cfg, seed=0)
+    ns = args.reference_tokens
+    x = batch.x[:ns].contiguous()
+    idx = batch.idx[:ns].contiguous()
+    w = batch.w[:ns].contiguous()
+    nb = sum(step_bytes(ns, cfg.H, cfg.k, cfg.E, cfg.R).values())
+    for _ in range(args.warmup):
+        oracle_sample_step(oracle, cfg, x, idx, w)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(oracle, cfg, x, idx, w)
+    el = time.perf_counter() - t0
+    value = nb * args.steps / el / 1e9
+    sample = (f"first {ns} tokens of the prefill batch per step (of {cfg.T}); "
+              f"single-threaded C oracle")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": ("prefill: T=4096 tokens, H=7168, E=256 experts in R=8 "
+                                    "logical ranks, top-8 group-limited routing; step = "
+                                    "layout + bf16 dispatch + FP8 dispatch + combine"),
+                       "sample_tokens_per_step": ns},
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--skip-decode", action="store_true")
+    p.add_argument("--skip-e2e", action="store_true")
+    p.add_argument("--skip-cpu", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--reference-tokens", type=int, default=256)
+    args = p.parse_args()
+    if args.warmup < 3:
+        p.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        res = bench_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    try:
+        res = bench_ours(args, world, rank, device)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+"""B200-native MoE expert-parallel dispatch/combine (DeepEP's hot path, with
+the ranks as logical partitions of one GPU's memory).
+
+Thin Python binding over the C ABI of ``libep.so`` (``include/ep.h``): it
+only marshals torch tensors (device memory and the current CUDA stream) into
+the C calls; every step runs in the library's CUDA kernels.  There is no
+CPU path: if the library is missing, calls raise ``EPLibraryError``.
+
+    layout = ep_get_layout(idx, E, R)                 # counts, offsets, rows
+    recv = ep_dispatch(x, layout.slot_pos)            # bf16 rows
+    q, scale = ep_dispatch(x, layout.slot_pos, fp8=True)
+    out = ep_combine(y, layout.slot_pos, w)           # gate-weighted sum
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+__all__ = ["EPError", "EPLibraryError", "Layout", "ep_get_layout",
+           "ep_dispatch", "ep_combine", "ep_read_error",
+           "ep_layout_workspace_bytes", "ep_kernel_launches", "lib",
+           "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_UNSUPPORTED", "EP_ERR_CUDA",
+           "EP_ERR_INDEX", "LIB_PATH"]
+
+EP_OK = 0
+EP_ERR_INVALID_ARG = 1
+EP_ERR_UNSUPPORTED = 2
+EP_ERR_CUDA = 3
+EP_ERR_INDEX = 4
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep.so")
+
+_lib = None
+
+
+class EPError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"[ep status {status}] {msg}")
+        self.status = status
+
+
+class EPLibraryError(ImportError):
+    pass
+
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+_SIGNATURES = {
+    "ep_abi_version": ([], _i),
+    "ep_last_error_string": ([], ctypes.c_char_p),
+    "ep_kernel_launches": ([], ctypes.c_uint64),
+    "ep_layout_workspace_bytes": ([_i, _i, _i, _i], _sz),
+    "ep_get_layout": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
+                       _vp, _vp, _sz, _vp, _vp], _i),
+    "ep_dispatch": ([_vp, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp], _i),
+    "ep_combine": ([_vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp], _i),
+    "ep_read_error": ([_vp, _vp], _i),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libep.so (raises EPLibraryError when it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise EPLibraryError(
+                f"{LIB_PATH} is missing; build it with "
+                "`python -m combine_ep_get_09_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != EP_OK:
+        raise EPError(status, lib().ep_last_error_string().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _need_cuda(name: str, t: torch.Tensor):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class Layout(NamedTuple):
+    cnt_e: torch.Tensor     # [E] int32
+    cnt_r: torch.Tensor     # [R] int32
+    in_rank: torch.Tensor   # [T, R] uint8
+    off_e: torch.Tensor     # [E+1] int32
+    off_r: torch.Tensor     # [R+1] int32
+    slot_pos: torch.Tensor  # [T, k] int32
+    recv_src: torch.Tensor  # [T*k] int32
+
+
+def ep_layout_workspace_bytes(T: int, k: int, E: int, R: int) -> int:
+    return int(lib().ep_layout_workspace_bytes(T, k, E, R))
+
+
+def ep_kernel_launches() -> int:
+    return int(lib().ep_kernel_launches())
+
+
+def empty_layout(T: int, k: int, E: int, R: int, device) -> Layout:
+    i32 = dict(dtype=torch.int32, device=device)
+    return Layout(torch.empty(E, **i32), torch.empty(R, **i32),
+                  torch.empty((T, R), dtype=torch.uint8, device=device),
+                  torch.empty(E + 1, **i32), torch.empty(R + 1, **i32),
+                  torch.empty((T, k), **i32), torch.empty(T * k, **i32))
+
+
+def ep_get_layout(idx: torch.Tensor, E: int, R: int, *,
+                  out: Optional[Layout] = None,
+                  ws: Optional[torch.Tensor] = None,
+                  d_err: Optional[torch.Tensor] = None,
+                  stream=None) -> Layout:
+    """Dispatch layout of expert ids ``idx`` [T, k] (int64 or int32, -1 =
+    dropped slot).  ``ws`` (uint8, zero-filled before first use, reused
+    across stream-ordered calls) is allocated zeroed when not given."""
+    _need_cuda("idx", idx)
+    if idx.dtype not in (torch.int64, torch.int32) or idx.dim() != 2:
+        raise ValueError("idx must be a 2-D int64 or int32 tensor")
+    T, k = idx.shape
+    if out is None:
+        out = empty_layout(T, k, E, R, idx.device)
+    need = ep_layout_workspace_bytes(T, k, E, R)
+    if ws is None and need > 0:
+        ws = torch.zeros(need, dtype=torch.uint8, device=idx.device)
+    _check(lib().ep_get_layout(
+        _ptr(idx), int(idx.dtype == torch.int64), T, k, E, R,
+        _ptr(out.cnt_e), _ptr(out.cnt_r), _ptr(out.in_rank), _ptr(out.off_e),
+        _ptr(out.off_r), _ptr(out.slot_pos), _ptr(out.recv_src),
+        _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _ptr(d_err), _stream(stream)))
+    return out
+
+
+def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
+                recv: Optional[torch.Tensor] = None,
+                recv_scale: Optional[torch.Tensor] = None,
+                num_sms: int = 0, stream=None):
+    """Rows of ``x`` [T, H] bf16 to their receive rows.  Returns ``recv``
+    [T*k, H] (bf16), or ``(recv_q [T*k, H] float8_e4m3fn, recv_scale
+    [T*k, H/128] fp32)`` when ``fp8``."""
+    _need_cuda("x", x)
+    _need_cuda("slot_pos", slot_pos)
+    if x.dtype != torch.bfloat16 or slot_pos.dtype != torch.int32:
+        raise ValueError("x must be bf16 and slot_pos int32")
+    T, H = x.shape
+    k = slot_pos.shape[1]
+    if recv is None:
+        recv = torch.empty((T * k, H), device=x.device,
+                           dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16)
+    if fp8 and recv_scale is None:
+        recv_scale = torch.empty((T * k, H // 128), device=x.device,
+                                 dtype=torch.float32)
+    _check(lib().ep_dispatch(_ptr(x), T, H, k, _ptr(slot_pos), int(bool(fp8)),
+                             _ptr(recv), _ptr(recv_scale) if fp8 else None,
+                             num_sms, _stream(stream)))
+    return (recv, recv_scale) if fp8 else recv
+
+
+def ep_combine(y: torch.Tensor, slot_pos: torch.Tensor, w: torch.Tensor, *,
+               out: Optional[torch.Tensor] = None, num_sms: int = 0,
+               stream=None) -> torch.Tensor:
+    """Gate-weighted combine of expert outputs ``y`` [T*k, H] bf16 into
+    ``out`` [T, H] bf16 (fp32 fma chain in slot order)."""
+    for name, t in (("y", y), ("slot_pos", slot_pos), ("w", w)):
+        _need_cuda(name, t)
+    if y.dtype != torch.bfloat16 or w.dtype != torch.float32:
+        raise ValueError("y must be bf16 and w fp32")
+    T, k = slot_pos.shape
+    H = y.shape[1]
+    if y.shape[0] < T * k:
+        raise ValueError(f"y needs at least T*k={T * k} rows")
+    if out is None:
+        out = torch.empty((T, H), device=y.device, dtype=torch.bfloat16)
+    _check(lib().ep_combine(_ptr(y), T, H, k, _ptr(slot_pos), _ptr(w),
+                            _ptr(out), num_sms, _stream(stream)))
+    return out
+
+
+def ep_read_error(d_err: torch.Tensor, stream=None) -> int:
+    """Waits for the stream and returns the device error word."""
+    st = lib().ep_read_error(_ptr(d_err), _stream(stream))
+    if st == EP_ERR_CUDA:
+        _check(st)
+    return int(st)

@@ -1,0 +1,178 @@
+// dispatch.cu -- token rows to expert-contiguous receive rows, as bf16 or
+// with the FP8 (e4m3, per-token per-128-channel fp32 scale) cast fused in.
+//
+// Both kernels are persistent grid-stride loops over work items
+// (token t, chunk c of its row).  A warp loads the chunk once with 128-bit
+// read-only streaming loads, then writes it to each of the token's k receive
+// rows with coalesced streaming stores, so HBM sees each source byte read
+// once and each destination byte written once.  The slot rows of the token
+// are fetched by lanes 0..k-1 and broadcast with shuffles.
+#include <cuda_fp8.h>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBf16Vec = 2;  // 16-byte vectors per lane per item (bf16 path)
+
+template <int V>
+__global__ void __launch_bounds__(kThreads)
+    dispatch_bf16_kernel(const uint4 *__restrict__ x, int T, int Hv, int k,
+                         const int32_t *__restrict__ slot_pos,
+                         uint4 *__restrict__ recv, long n_rows) {
+  const int lane = threadIdx.x & 31;
+  const int per_chunk = 32 * V;
+  const int nchunks = (Hv + per_chunk - 1) / per_chunk;
+  const long items = static_cast<long>(T) * nchunks;
+  const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
+  for (long it = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       it < items; it += nwarps) {
+    const int t = static_cast<int>(it / nchunks);
+    const int c = static_cast<int>(it - static_cast<long>(t) * nchunks);
+    const int sp = lane < k ? __ldg(slot_pos + static_cast<long>(t) * k + lane) : -1;
+    const int v0 = c * per_chunk + lane;
+    const uint4 *src = x + static_cast<long>(t) * Hv;
+    uint4 v[V];
+#pragma unroll
+    for (int u = 0; u < V; ++u)
+      v[u] = v0 + 32 * u < Hv ? ld_stream_v4(src + v0 + 32 * u) : make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < k; ++j) {
+      const int row = __shfl_sync(0xffffffffu, sp, j);
+      if (row < 0 || row >= n_rows) continue;  // uniform across the warp
+      uint4 *dst = recv + static_cast<long>(row) * Hv;
+#pragma unroll
+      for (int u = 0; u < V; ++u)
+        if (v0 + 32 * u < Hv) st_stream_v4(dst + v0 + 32 * u, v[u]);
+    }
+  }
+}
+
+// Largest |value| of 8 bf16 values as a bf16 bit pattern: with the sign
+// cleared, bf16 bit patterns order like their magnitudes (NaN above inf), so
+// an unsigned max of the patterns is the max of |x| with NaN propagating.
+__device__ __forceinline__ uint32_t absmax_bits_bf16x8(uint4 v) {
+  const uint32_t a = __vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu);
+  const uint32_t b = __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu);
+  const uint32_t m = __vmaxu2(a, b);
+  return max(m & 0xffffu, m >> 16);
+}
+
+// e4m3 codes of x / s for 8 bf16 values: IEEE fp32 quotient (round to
+// nearest), then the hardware e4m3 conversion (round to nearest even,
+// saturating to +-448).
+__device__ __forceinline__ uint2 quantize_bf16x8(uint4 v, float s) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __uint_as_float(in[i] << 16);
+    const float hi = __uint_as_float(in[i] & 0xffff0000u);
+    q[i] = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(lo, s), __fdiv_rn(hi, s)),
+                                    __NV_SATFINITE, __NV_E4M3);
+  }
+  return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+}
+
+// Work item = (token, chunk of 4 blocks of 128 channels).  Lane l covers
+// 8 channels of block 2p + (l >> 4) for p = 0, 1: each half-warp owns a
+// block per load, so the amax reduction is 4 xor-shuffles inside it and
+// every load / store instruction of the warp touches one contiguous span.
+__global__ void __launch_bounds__(kThreads)
+    dispatch_fp8_kernel(const uint4 *__restrict__ x, int T, int H, int k,
+                        const int32_t *__restrict__ slot_pos,
+                        uint2 *__restrict__ recv_q,
+                        float *__restrict__ recv_scale, long n_rows) {
+  const int lane = threadIdx.x & 31, half = lane >> 4, sub = lane & 15;
+  const int Hv = H >> 3;   // 8-channel units per row (16 B in, 8 B out)
+  const int nb = H >> 7;   // 128-channel blocks per row
+  const int nchunks = (nb + 3) >> 2;
+  const long items = static_cast<long>(T) * nchunks;
+  const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
+  for (long it = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       it < items; it += nwarps) {
+    const int t = static_cast<int>(it / nchunks);
+    const int c = static_cast<int>(it - static_cast<long>(t) * nchunks);
+    const int sp = lane < k ? __ldg(slot_pos + static_cast<long>(t) * k + lane) : -1;
+    const uint4 *src = x + static_cast<long>(t) * Hv;
+
+    int blk[2];
+    bool ok[2];
+    uint4 v[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      blk[p] = 4 * c + 2 * p + half;
+      ok[p] = blk[p] < nb;
+      v[p] = ok[p] ? ld_stream_v4(src + blk[p] * 16 + sub) : make_uint4(0, 0, 0, 0);
+    }
+    float s[2];
+    uint2 q[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      uint32_t m = absmax_bits_bf16x8(v[p]);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float a = __uint_as_float(m << 16);
+      a = a < 1e-4f ? 1e-4f : a;  // keeps NaN
+      s[p] = __fdiv_rn(a, 448.0f);
+      q[p] = quantize_bf16x8(v[p], s[p]);
+    }
+    for (int j = 0; j < k; ++j) {
+      const int row = __shfl_sync(0xffffffffu, sp, j);
+      if (row < 0 || row >= n_rows) continue;
+      uint2 *dst = recv_q + static_cast<long>(row) * Hv;
+#pragma unroll
+      for (int p = 0; p < 2; ++p)
+        if (ok[p]) st_stream_v2(dst + blk[p] * 16 + sub, q[p]);
+    }
+    // scales: lane l stores block (l & 3) of the chunk for slot j0 + (l >> 2);
+    // block 2p + h's scale sits in s[p] of half h
+    const int bb = lane & 3;
+    const float s0 = __shfl_sync(0xffffffffu, s[0], (bb & 1) * 16);
+    const float s1 = __shfl_sync(0xffffffffu, s[1], (bb & 1) * 16);
+    const float sv = (bb >> 1) ? s1 : s0;
+    const int b = 4 * c + bb;
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      const int j = j0 + (lane >> 2);
+      const int row = __shfl_sync(0xffffffffu, sp, j & 31);
+      if (j < k && b < nb && row >= 0 && row < n_rows)
+        st_stream_f32(recv_scale + static_cast<long>(row) * nb + b, sv);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
+                                 const int32_t *slot_pos, void *recv,
+                                 int num_sms, cudaStream_t s, int *launches) {
+  const int Hv = H / 8;
+  const long nchunks = (Hv + 32 * kBf16Vec - 1) / (32 * kBf16Vec);
+  const long items = static_cast<long>(T) * nchunks;
+  if (items == 0) return cudaSuccess;
+  auto kern = dispatch_bf16_kernel<kBf16Vec>;
+  const long grid = persistent_grid(reinterpret_cast<const void *>(kern), kThreads, items, num_sms);
+  kern<<<grid, kThreads, 0, s>>>(static_cast<const uint4 *>(x), T, Hv, k, slot_pos,
+                                 static_cast<uint4 *>(recv), static_cast<long>(T) * k);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
+                                const int32_t *slot_pos, void *recv_q,
+                                float *recv_scale, int num_sms,
+                                cudaStream_t s, int *launches) {
+  const long nchunks = (H / 128 + 3) / 4;
+  const long items = static_cast<long>(T) * nchunks;
+  if (items == 0) return cudaSuccess;
+  const long grid = persistent_grid(reinterpret_cast<const void *>(dispatch_fp8_kernel),
+                                    kThreads, items, num_sms);
+  dispatch_fp8_kernel<<<grid, kThreads, 0, s>>>(
+      static_cast<const uint4 *>(x), T, H, k, slot_pos, static_cast<uint2 *>(recv_q),
+      recv_scale, static_cast<long>(T) * k);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+}  // namespace ep

@@ -1,0 +1,238 @@
+// ep_abi.cu -- the extern "C" entry points of libep.so: argument checks,
+// launch, error reporting.  Every check happens before anything is
+// enqueued; the kernels themselves live in layout.cu, dispatch.cu and
+// combine.cu.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "ep_internal.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+std::atomic<uint64_t> g_launches{0};
+
+ep_status_t fail(ep_status_t st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+ep_status_t from_cuda(cudaError_t e, const char *where) {
+  if (e == cudaSuccess) return EP_OK;
+  return fail(EP_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorString(e),
+              cudaGetErrorName(e));
+}
+
+bool aligned(const void *p, size_t a) {
+  return reinterpret_cast<uintptr_t>(p) % a == 0;
+}
+
+// Shared size checks of dispatch and combine.
+ep_status_t check_rows(const char *fn, int T, int H, int k, int num_sms) {
+  if (T < 0) return fail(EP_ERR_INVALID_ARG, "%s: T=%d < 0", fn, T);
+  if (H <= 0) return fail(EP_ERR_INVALID_ARG, "%s: H=%d <= 0", fn, H);
+  if (k < 1) return fail(EP_ERR_INVALID_ARG, "%s: k=%d < 1", fn, k);
+  if (num_sms < 0) return fail(EP_ERR_INVALID_ARG, "%s: num_sms=%d < 0", fn, num_sms);
+  if (k > EP_MAX_K)
+    return fail(EP_ERR_UNSUPPORTED, "%s: k=%d > %d", fn, k, EP_MAX_K);
+  if (H % 8 != 0)
+    return fail(EP_ERR_UNSUPPORTED, "%s: H=%d is not a multiple of 8", fn, H);
+  if (static_cast<long long>(T) * k > 0x7fffffffLL)
+    return fail(EP_ERR_UNSUPPORTED, "%s: T*k=%lld does not fit int32", fn,
+                static_cast<long long>(T) * k);
+  return EP_OK;
+}
+
+#define EP_REQUIRE_PTR(fn, p, align)                                          \
+  do {                                                                        \
+    if ((p) == nullptr)                                                       \
+      return fail(EP_ERR_INVALID_ARG, "%s: %s is NULL", fn, #p);              \
+    if (!aligned((p), (align)))                                               \
+      return fail(EP_ERR_INVALID_ARG, "%s: %s is not %d-byte aligned", fn, #p, \
+                  static_cast<int>(align));                                   \
+  } while (0)
+
+}  // namespace
+
+namespace ep {
+
+int device_sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    n = 1;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+long persistent_grid(const void *kernel, int threads, long items, int num_sms) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void *>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int per_sm = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find({dev, kernel});
+    if (it != cache.end()) {
+      per_sm = it->second;
+    } else {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) !=
+              cudaSuccess ||
+          per_sm < 1)
+        per_sm = 1;
+      cache[{dev, kernel}] = per_sm;
+    }
+  }
+  const int sms = num_sms > 0 ? num_sms : device_sm_count();
+  const long warps_per_block = threads / kWarp;
+  const long need = (items + warps_per_block - 1) / warps_per_block;
+  const long cap = static_cast<long>(sms) * per_sm;
+  return need < cap ? need : cap;
+}
+
+}  // namespace ep
+
+extern "C" {
+
+int ep_abi_version(void) { return 1; }
+
+const char *ep_last_error_string(void) { return g_err; }
+
+uint64_t ep_kernel_launches(void) { return g_launches.load(); }
+
+static ep_status_t check_layout_sizes(const char *fn, int T, int k, int E, int R) {
+  if (T < 0) return fail(EP_ERR_INVALID_ARG, "%s: T=%d < 0", fn, T);
+  if (k < 1) return fail(EP_ERR_INVALID_ARG, "%s: k=%d < 1", fn, k);
+  if (E < 1) return fail(EP_ERR_INVALID_ARG, "%s: E=%d < 1", fn, E);
+  if (R < 1) return fail(EP_ERR_INVALID_ARG, "%s: R=%d < 1", fn, R);
+  if (E % R != 0)
+    return fail(EP_ERR_INVALID_ARG, "%s: E=%d is not a multiple of R=%d", fn, E, R);
+  if (k > E) return fail(EP_ERR_INVALID_ARG, "%s: k=%d > E=%d", fn, k, E);
+  if (k > EP_MAX_K) return fail(EP_ERR_UNSUPPORTED, "%s: k=%d > %d", fn, k, EP_MAX_K);
+  if (E > EP_MAX_E) return fail(EP_ERR_UNSUPPORTED, "%s: E=%d > %d", fn, E, EP_MAX_E);
+  if (R > EP_MAX_R) return fail(EP_ERR_UNSUPPORTED, "%s: R=%d > %d", fn, R, EP_MAX_R);
+  if (static_cast<long long>(T) * k > 0x7fffffffLL)
+    return fail(EP_ERR_UNSUPPORTED, "%s: T*k does not fit int32", fn);
+  return EP_OK;
+}
+
+size_t ep_layout_workspace_bytes(int T, int k, int E, int R) {
+  if (check_layout_sizes("ep_layout_workspace_bytes", T, k, E, R) != EP_OK) return 0;
+  return ep::layout_workspace_bytes(T, k, E, R);
+}
+
+ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
+                          int E, int R, int32_t *cnt_e, int32_t *cnt_r,
+                          uint8_t *in_rank, int32_t *off_e, int32_t *off_r,
+                          int32_t *slot_pos, int32_t *recv_src, void *ws,
+                          size_t ws_bytes, int32_t *d_err, void *stream) {
+  static const char fn[] = "ep_get_layout";
+  g_err[0] = '\0';
+  ep_status_t st = check_layout_sizes(fn, T, k, E, R);
+  if (st != EP_OK) return st;
+  EP_REQUIRE_PTR(fn, cnt_e, 4);
+  EP_REQUIRE_PTR(fn, cnt_r, 4);
+  EP_REQUIRE_PTR(fn, off_e, 4);
+  EP_REQUIRE_PTR(fn, off_r, 4);
+  if (T > 0) {
+    EP_REQUIRE_PTR(fn, idx, idx_is_int64 ? 8 : 4);
+    EP_REQUIRE_PTR(fn, in_rank, 1);
+    EP_REQUIRE_PTR(fn, slot_pos, 4);
+    EP_REQUIRE_PTR(fn, recv_src, 4);
+  }
+  if (d_err != nullptr && !aligned(d_err, 4))
+    return fail(EP_ERR_INVALID_ARG, "%s: d_err is not 4-byte aligned", fn);
+  const size_t need = ep::layout_workspace_bytes(T, k, E, R);
+  if (need > 0) {
+    EP_REQUIRE_PTR(fn, ws, 16);
+    if (ws_bytes < need)
+      return fail(EP_ERR_INVALID_ARG, "%s: ws_bytes=%zu < %zu needed", fn, ws_bytes, need);
+  }
+  ep::LayoutArgs a{};
+  a.idx = idx;
+  a.idx_is_int64 = idx_is_int64 ? 1 : 0;
+  a.T = T;
+  a.k = k;
+  a.E = E;
+  a.R = R;
+  a.cnt_e = cnt_e;
+  a.cnt_r = cnt_r;
+  a.off_e = off_e;
+  a.off_r = off_r;
+  a.slot_pos = slot_pos;
+  a.recv_src = recv_src;
+  a.in_rank = in_rank;
+  a.ws = ws;
+  a.d_err = d_err;
+  int n = 0;
+  const cudaError_t e = ep::launch_layout(a, static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
+  return from_cuda(e, fn);
+}
+
+ep_status_t ep_dispatch(const void *x, int T, int H, int k,
+                        const int32_t *slot_pos, int fp8, void *recv,
+                        float *recv_scale, int num_sms, void *stream) {
+  static const char fn[] = "ep_dispatch";
+  g_err[0] = '\0';
+  ep_status_t st = check_rows(fn, T, H, k, num_sms);
+  if (st != EP_OK) return st;
+  if (fp8 && H % 128 != 0)
+    return fail(EP_ERR_UNSUPPORTED, "%s: fp8 needs H %% 128 == 0 (H=%d)", fn, H);
+  if (T == 0) return EP_OK;
+  EP_REQUIRE_PTR(fn, x, 16);
+  EP_REQUIRE_PTR(fn, slot_pos, 4);
+  EP_REQUIRE_PTR(fn, recv, 16);
+  if (fp8) EP_REQUIRE_PTR(fn, recv_scale, 4);
+  int n = 0;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e =
+      fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale, num_sms, s, &n)
+          : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, num_sms, s, &n);
+  g_launches += n;
+  return from_cuda(e, fn);
+}
+
+ep_status_t ep_combine(const void *y, int T, int H, int k,
+                       const int32_t *slot_pos, const float *w, void *out,
+                       int num_sms, void *stream) {
+  static const char fn[] = "ep_combine";
+  g_err[0] = '\0';
+  ep_status_t st = check_rows(fn, T, H, k, num_sms);
+  if (st != EP_OK) return st;
+  if (T == 0) return EP_OK;
+  EP_REQUIRE_PTR(fn, y, 16);
+  EP_REQUIRE_PTR(fn, slot_pos, 4);
+  EP_REQUIRE_PTR(fn, w, 4);
+  EP_REQUIRE_PTR(fn, out, 16);
+  int n = 0;
+  const cudaError_t e = ep::launch_combine(y, T, H, k, slot_pos, w, out, num_sms,
+                                           static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
+  return from_cuda(e, fn);
+}
+
+ep_status_t ep_read_error(const int32_t *d_err, void *stream) {
+  static const char fn[] = "ep_read_error";
+  g_err[0] = '\0';
+  EP_REQUIRE_PTR(fn, d_err, 4);
+  int32_t h = 0;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&h, d_err, sizeof h, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return from_cuda(e, fn);
+  return h;
+}
+
+}  // extern "C"

@@ -1,0 +1,88 @@
+// ep_internal.cuh -- device helpers and launcher declarations shared by the
+// kernels of libep.so (internal; the public ABI is include/ep.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep.h"
+
+namespace ep {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------- memory
+
+// 128-bit read-only load that bypasses L1 allocation: the row is read once
+// per launch, so keeping it out of L1 leaves L1 to the index arrays.  The
+// DeepEP blog (frogred8, "deepEP optimization", second method) describes
+// the same non-coherent, no-allocate read for its communication buffers.
+__device__ __forceinline__ uint4 ld_stream_v4(const uint4 *p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+// Write-once outputs: streaming stores (evict-first in L1 and L2).
+__device__ __forceinline__ void st_stream_v4(uint4 *p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_stream_v2(uint2 *p, uint2 v) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x),
+               "r"(v.y)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_stream_f32(float *p, float v) {
+  asm volatile("st.global.cs.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// --------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error; arguments are validated by
+// the ABI layer before these are called.
+
+struct LayoutArgs {
+  const void *idx;
+  int idx_is_int64;
+  int T, k, E, R;
+  int32_t *cnt_e, *cnt_r, *off_e, *off_r, *slot_pos, *recv_src;
+  uint8_t *in_rank;
+  void *ws;
+  int32_t *d_err;
+};
+
+size_t layout_workspace_bytes(int T, int k, int E, int R);
+cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s, int *launches);
+
+cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
+                                 const int32_t *slot_pos, void *recv,
+                                 int num_sms, cudaStream_t s, int *launches);
+cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
+                                const int32_t *slot_pos, void *recv_q,
+                                float *recv_scale, int num_sms,
+                                cudaStream_t s, int *launches);
+cudaError_t launch_combine(const void *y, int T, int H, int k,
+                           const int32_t *slot_pos, const float *w, void *out,
+                           int num_sms, cudaStream_t s, int *launches);
+
+// SM count of the current device (cached per device).
+int device_sm_count();
+
+// Grid for a persistent grid-stride kernel: enough blocks of `threads`
+// threads (warps_per_item = 1) to cover `items` warp work items, capped at
+// the blocks that fit at once on `num_sms` SMs (0 = all SMs).  The
+// occupancy figure is cached per (device, kernel).
+long persistent_grid(const void *kernel, int threads, long items, int num_sms);
+
+}  // namespace ep

@@ -1,0 +1,171 @@
+/*
+ * ep.h -- C ABI of the B200 (sm_100a) MoE expert-parallel dispatch/combine
+ * library (libep.so).
+ *
+ * The operation is DeepEP's: route every token to the experts of its top-k
+ * choice and bring the expert outputs back ("all-to-all" dispatch and
+ * combine for MoE, with native FP8 dispatch -- chinainews.com, "DeepSeek
+ * releases DeepEP", feature list; Wallstreetcn/lbkrs review, feature list;
+ * dataforcee.us rewrite, "Technological Views and Benefits": tokens are
+ * "shipped and combined" across experts).  Here the expert-parallel ranks
+ * are logical partitions of one GPU's memory: rank r owns the G = E / R
+ * consecutive experts [r*G, (r+1)*G), and "sending to rank r" means writing
+ * into rank r's segment of one expert-contiguous receive buffer.
+ *
+ * Notation: T tokens, hidden size H, top-k slots per token, E experts,
+ * R ranks.  idx[T,k] expert ids (-1 = dropped slot), w[T,k] fp32 gate
+ * weights, x[T,H] bf16 hidden states.  N = T*k is the receive capacity.
+ * All arrays are dense row-major in device memory unless stated otherwise.
+ *
+ * Conventions for every entry point:
+ *  - Asynchronous: work is enqueued on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) and the call returns without waiting.
+ *  - Stateless: nothing is kept between calls, so calls on different
+ *    streams with different buffers may run concurrently.
+ *  - The caller allocates and owns every buffer; the library allocates no
+ *    device memory.
+ *  - Argument errors are returned before anything is enqueued; nothing is
+ *    written then.  EP_ERR_CUDA means a launch failed; the message is in
+ *    ep_last_error_string().  Nothing ever traps on the device: a bad
+ *    expert id found on the device is written to *d_err (EP_ERR_INDEX) and
+ *    its slot is treated as dropped.
+ *  - Pointers must be 16-byte aligned unless stated otherwise.
+ */
+#ifndef EP_H_
+#define EP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int ep_status_t;
+
+#define EP_OK 0
+#define EP_ERR_INVALID_ARG 1 /* null/misaligned pointer, bad size        */
+#define EP_ERR_UNSUPPORTED 2 /* valid request outside the built limits   */
+#define EP_ERR_CUDA 3        /* a CUDA call failed; see ep_last_error_string */
+#define EP_ERR_INDEX 4       /* device-side: an expert id outside [-1, E) */
+
+#define EP_MAX_K 32    /* top-k slots per token            */
+#define EP_MAX_E 1024  /* experts                          */
+#define EP_MAX_R 64    /* logical ranks                    */
+
+/* Version of this ABI (incremented on any signature change). */
+int ep_abi_version(void);
+
+/* Message of the last error returned on this host thread ("" if none). */
+const char *ep_last_error_string(void);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t ep_kernel_launches(void);
+
+/*
+ * Bytes of device workspace ep_get_layout needs for (T, k, E, R); 0 when the
+ * single-block path applies (then ws may be NULL).
+ */
+size_t ep_layout_workspace_bytes(int T, int k, int E, int R);
+
+/*
+ * ep_get_layout -- the dispatch layout: who goes where.
+ *
+ * The pages describe per-rank senders that each push a token to every
+ * peer rank that needs it (frogred8 blog, "Implementation of SMs dedicated
+ * to network communication": warp roles per peer, up to 8 NVLink peers),
+ * which presumes per-rank counts, a token-in-rank mask and the prefix
+ * offsets computed here; the layout follows the group-limited gating of
+ * DeepSeek-V3 that DeepEP targets (chinainews.com item, paragraph on the
+ * V3 paper).  Definitions (the pages give none; this is the reading):
+ *   cnt_e[E]     number of slots (t,j) with idx[t,j] == e
+ *   off_e[E+1]   exclusive prefix sum of cnt_e; off_e[E] = kept slots
+ *   slot_pos[T,k] receive row of slot (t,j): off_e[e] + number of slots
+ *                before (t,j) in token-major order with the same expert
+ *                (stable: rows of one expert are in ascending token order);
+ *                -1 for dropped slots
+ *   recv_src[N]  token whose copy lands in each row; -1 past off_e[E]
+ *   in_rank[T,R] (uint8) 1 iff token t has a kept slot in rank r's experts
+ *   cnt_r[R]     tokens per rank (sum over t of in_rank[t,r])
+ *   off_r[R+1]   exclusive prefix sum of cnt_r
+ * Rank r's rows are [off_e[r*G], off_e[(r+1)*G]).
+ *
+ * idx          [T,k] int64 (idx_is_int64 != 0) or int32 expert ids; -1 drops
+ *              a slot.  8-byte (int64) or 4-byte (int32) aligned.
+ * T >= 0, 1 <= k <= min(E, EP_MAX_K), 1 <= E <= EP_MAX_E,
+ * 1 <= R <= EP_MAX_R, E % R == 0, T*k < 2^31.
+ * Outputs: int32 arrays 4-byte aligned, in_rank 1-byte aligned.
+ * ws, ws_bytes  device scratch of at least ep_layout_workspace_bytes()
+ *              bytes, 16-byte aligned.  It must be zero-filled before its
+ *              first use; every call leaves it zero-filled again, so one
+ *              buffer serves a sequence of stream-ordered calls (not
+ *              concurrent ones).
+ * d_err        optional (may be NULL) device int32; set to EP_ERR_INDEX when
+ *              an id outside [-1, E) is met (that slot is then dropped).
+ *              Never cleared by the library.
+ * Returns EP_OK, EP_ERR_INVALID_ARG, EP_ERR_UNSUPPORTED or EP_ERR_CUDA.
+ */
+ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
+                          int E, int R, int32_t *cnt_e, int32_t *cnt_r,
+                          uint8_t *in_rank, int32_t *off_e, int32_t *off_r,
+                          int32_t *slot_pos, int32_t *recv_src, void *ws,
+                          size_t ws_bytes, int32_t *d_err, void *stream);
+
+/*
+ * ep_dispatch -- send each token to its experts' receive rows.
+ *
+ * DeepEP's dispatch (chinainews.com item, feature list: "all-to-all" for
+ * MoE, native FP8 support; Wallstreetcn/lbkrs review: "Native FP8 dispatch
+ * support"; frogred8 blog, TMA bulk copies and read-only non-coherent
+ * loads).  For every slot (t,j) with slot_pos[t,j] = p >= 0:
+ *   fp8 == 0:  recv[p, :] = x[t, :]                    (bf16 rows)
+ *   fp8 != 0:  per 128-channel block b of token t,
+ *              a = max |x[t, 128b : 128b+128]| (NaN propagates),
+ *              a = max(a, 1e-4); s = a / 448 (fp32, round to nearest);
+ *              recv[p, c] = e4m3(x[t, c] / s)  (fp32 quotient rounded to
+ *              nearest; e4m3 round-to-nearest-even, saturating to +-448;
+ *              NaN -> 0x7f);  recv_scale[p, b] = s.
+ * x           [T,H] bf16.
+ * slot_pos    [T,k] int32 from ep_get_layout; values outside [0, T*k) are
+ *             skipped.
+ * recv        [T*k, H] bf16 (fp8 == 0) or e4m3 bytes (fp8 != 0).  Rows no
+ *             slot points at are left untouched.
+ * recv_scale  [T*k, H/128] fp32 (fp8 != 0, 4-byte aligned), else ignored.
+ * T >= 0, 1 <= k <= EP_MAX_K, H > 0 with H % 8 == 0 (H % 128 == 0 for
+ * fp8), T*k < 2^31.
+ * num_sms     SMs to spread the work over (0 = all of them).
+ */
+ep_status_t ep_dispatch(const void *x, int T, int H, int k,
+                        const int32_t *slot_pos, int fp8, void *recv,
+                        float *recv_scale, int num_sms, void *stream);
+
+/*
+ * ep_combine -- bring the expert outputs back to their tokens.
+ *
+ * DeepEP's combine (chinainews.com item, feature list; dataforcee.us
+ * rewrite, "Technological Views and Benefits").  Reading: a gate-weighted
+ * sum accumulated in fp32 in slot order:
+ *   acc = 0.0f;  for j = 0..k-1 with slot_pos[t,j] = p >= 0:
+ *       acc = fma(w[t,j], float(y[p, :]), acc)
+ *   out[t, :] = bf16 round-to-nearest-even(acc)
+ * y          [T*k, H] bf16 expert outputs in receive-row order.
+ * slot_pos   [T,k] int32; values outside [0, T*k) are skipped.
+ * w          [T,k] fp32 gate weights (4-byte aligned).
+ * out        [T,H] bf16; a token with no kept slot gets +0.
+ * Limits as ep_dispatch (H % 8 == 0).
+ */
+ep_status_t ep_combine(const void *y, int T, int H, int k,
+                       const int32_t *slot_pos, const float *w, void *out,
+                       int num_sms, void *stream);
+
+/*
+ * Waits for `stream` and returns the device error word *d_err (EP_OK when
+ * no bad id was met), or EP_ERR_CUDA if the copy failed.
+ */
+ep_status_t ep_read_error(const int32_t *d_err, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_H_ */

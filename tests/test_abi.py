@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/ep.h declares, and rejects bad arguments before
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_ep_get_09_b200 as ep
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "ep.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ep_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert "ep_get_layout" in names and "ep_dispatch" in names and "ep_combine" in names
+    L = ctypes.CDLL(ep.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) <= set(ep._SIGNATURES), "binding lacks a declared symbol"
+
+
+def test_abi_version():
+    assert ep.lib().ep_abi_version() == 1
+
+
+def test_workspace_sizes():
+    # single-block path needs none; the tiled path one row of E + R counts
+    # per tile plus a 16-byte ticket
+    assert ep.ep_layout_workspace_bytes(128, 8, 256, 8) == 0
+    assert ep.ep_layout_workspace_bytes(0, 8, 256, 8) == 0
+    assert ep.ep_layout_workspace_bytes(4096, 8, 256, 8) == 16 + 32 * 264 * 4
+    assert ep.ep_layout_workspace_bytes(32768, 8, 128, 16) == 16 + 256 * 144 * 4
+    # invalid sizes report 0
+    assert ep.ep_layout_workspace_bytes(4096, 8, 250, 8) == 0
+
+
+def _layout_call(**kw):
+    a = dict(idx=16, idx_is_int64=1, T=4, k=2, E=8, R=2, cnt_e=16, cnt_r=16,
+             in_rank=16, off_e=16, off_r=16, slot_pos=16, recv_src=16, ws=None,
+             ws_bytes=0, d_err=None, stream=None)
+    a.update(kw)
+    return ep.lib().ep_get_layout(*a.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=-1), ep.EP_ERR_INVALID_ARG),
+    (dict(k=0), ep.EP_ERR_INVALID_ARG),
+    (dict(E=0), ep.EP_ERR_INVALID_ARG),
+    (dict(R=0), ep.EP_ERR_INVALID_ARG),
+    (dict(E=9), ep.EP_ERR_INVALID_ARG),          # E % R != 0
+    (dict(k=9), ep.EP_ERR_INVALID_ARG),          # k > E
+    (dict(k=33, E=64), ep.EP_ERR_UNSUPPORTED),
+    (dict(E=2048), ep.EP_ERR_UNSUPPORTED),
+    (dict(E=128, R=128), ep.EP_ERR_UNSUPPORTED),
+    (dict(T=1 << 30, k=4), ep.EP_ERR_UNSUPPORTED),
+    (dict(cnt_e=None), ep.EP_ERR_INVALID_ARG),
+    (dict(idx=None), ep.EP_ERR_INVALID_ARG),
+    (dict(idx=20), ep.EP_ERR_INVALID_ARG),       # int64 ids need 8-byte alignment
+    (dict(slot_pos=18), ep.EP_ERR_INVALID_ARG),
+    (dict(T=4096, k=8, E=256, R=8), ep.EP_ERR_INVALID_ARG),   # tiled path, no ws
+    (dict(T=4096, k=8, E=256, R=8, ws=16, ws_bytes=100), ep.EP_ERR_INVALID_ARG),
+    (dict(T=4096, k=8, E=256, R=8, ws=24, ws_bytes=1 << 20), ep.EP_ERR_INVALID_ARG),
+])
+def test_layout_rejects(kw, status):
+    assert _layout_call(**kw) == status
+    assert ep.lib().ep_last_error_string().decode()
+
+
+@pytest.mark.parametrize("args,status", [
+    ((16, -1, 64, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 0, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 12, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_UNSUPPORTED),   # H % 8
+    ((16, 4, 64, 2, 16, 1, 16, 16, 0, None), ep.EP_ERR_UNSUPPORTED),     # fp8, H % 128
+    ((16, 4, 64, 33, 16, 0, 16, None, 0, None), ep.EP_ERR_UNSUPPORTED),  # k > 32
+    ((16, 4, 64, 2, 16, 0, 16, None, -1, None), ep.EP_ERR_INVALID_ARG),  # num_sms
+    ((None, 4, 64, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
+    ((24, 4, 64, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),   # x misaligned
+    ((16, 4, 128, 2, 16, 1, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),  # fp8, no scale
+    ((16, 4, 64, 2, 16, 0, 8, None, 0, None), ep.EP_ERR_INVALID_ARG),    # recv misaligned
+])
+def test_dispatch_rejects(args, status):
+    assert ep.lib().ep_dispatch(*args) == status
+
+
+def test_dispatch_combine_empty_batch_is_a_no_op():
+    # T = 0: valid, nothing to do, nothing touched (no device needed)
+    assert ep.lib().ep_dispatch(None, 0, 64, 2, None, 0, None, None, 0, None) == ep.EP_OK
+    assert ep.lib().ep_combine(None, 0, 64, 2, None, None, None, 0, None) == ep.EP_OK
+
+
+@pytest.mark.parametrize("args,status", [
+    ((16, 4, 64, 2, 16, None, 16, 0, None), ep.EP_ERR_INVALID_ARG),  # no w
+    ((16, 4, 64, 2, 16, 18, 16, 0, None), ep.EP_ERR_INVALID_ARG),    # w misaligned
+    ((16, 4, 60, 2, 16, 16, 16, 0, None), ep.EP_ERR_UNSUPPORTED),
+    ((16, 4, 64, 2, 16, 16, 40, 0, None), ep.EP_ERR_INVALID_ARG),    # out misaligned
+])
+def test_combine_rejects(args, status):
+    assert ep.lib().ep_combine(*args) == status
+
+
+def test_read_error_rejects_null():
+    assert ep.lib().ep_read_error(None, None) == ep.EP_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(ep, "_lib", None)
+    monkeypatch.setattr(ep, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ep.EPLibraryError):
+        ep.lib()

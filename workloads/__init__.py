@@ -183,16 +183,19 @@ def expert_outputs(x: torch.Tensor, recv_src: torch.Tensor,
     src = recv_src.to(torch.int64)
     n = src.numel()
     y = torch.zeros((n, x.shape[1]), dtype=torch.bfloat16, device=x.device)
-    valid = src >= 0
-    if not bool(valid.any()):
-        return y
-    rows = x[src[valid]]
-    if kind == "identity":
-        y[valid] = rows
-    elif kind == "scale":
-        e = row_experts(off_e, n)[valid].to(torch.float32)
-        f = 1.0 + 0.01 * e
-        y[valid] = (rows.to(torch.float32) * f[:, None]).to(torch.bfloat16)
-    else:
+    if kind not in ("identity", "scale"):
         raise ValueError(f"unknown expert kind {kind!r}")
+    e_all = row_experts(off_e.to(x.device), n) if kind == "scale" else None
+    step = 1 << 16  # rows per chunk: bounds the fp32 temporaries
+    for r0 in range(0, n, step):
+        s = src[r0:r0 + step]
+        valid = s >= 0
+        if not bool(valid.any()):
+            continue
+        rows = x[s[valid]]
+        if kind == "identity":
+            y[r0:r0 + step][valid] = rows
+        else:
+            f = 1.0 + 0.01 * e_all[r0:r0 + step][valid].to(torch.float32)
+            y[r0:r0 + step][valid] = (rows.to(torch.float32) * f[:, None]).to(torch.bfloat16)
     return y
