@@ -20,6 +20,7 @@ from typing import NamedTuple, Optional
 import torch
 
 __all__ = ["EPError", "EPLibraryError", "Layout", "ep_get_layout",
+           "ep_get_layout_noalloc", "EP_NOALLOC_SCRATCH_BYTES",
            "ep_dispatch", "ep_combine", "ep_read_error",
            "ep_layout_workspace_bytes", "ep_kernel_launches", "lib",
            "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_UNSUPPORTED", "EP_ERR_CUDA",
@@ -30,6 +31,7 @@ EP_ERR_INVALID_ARG = 1
 EP_ERR_UNSUPPORTED = 2
 EP_ERR_CUDA = 3
 EP_ERR_INDEX = 4
+EP_NOALLOC_SCRATCH_BYTES = 256 * 1024
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep.so")
 
@@ -60,6 +62,8 @@ _SIGNATURES = {
     "ep_dispatch": ([_vp, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp], _i),
     "ep_combine": ([_vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp], _i),
     "ep_read_error": ([_vp, _vp], _i),
+    "ep_get_layout_noalloc": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                               _vp, _vp, _vp, _vp], _i),
 }
 
 
@@ -152,6 +156,30 @@ def ep_get_layout(idx: torch.Tensor, E: int, R: int, *,
         _ptr(out.cnt_e), _ptr(out.cnt_r), _ptr(out.in_rank), _ptr(out.off_e),
         _ptr(out.off_r), _ptr(out.slot_pos), _ptr(out.recv_src),
         _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _ptr(d_err), _stream(stream)))
+    return out
+
+
+def ep_get_layout_noalloc(idx: torch.Tensor, E: int, R: int, *,
+                          out: Optional[Layout] = None,
+                          d_err: Optional[torch.Tensor] = None,
+                          stream=None) -> Layout:
+    """ep_get_layout for callers that cannot allocate device memory: the
+    library's fixed scratch array (EP_NOALLOC_SCRATCH_BYTES per device)
+    replaces the workspace.  Calls that overlap on the GPU race on that
+    array; the first call on a device looks its address up, so make it
+    before any stream capture.  Outputs are allocated here only when
+    ``out`` is not given."""
+    _need_cuda("idx", idx)
+    if idx.dtype not in (torch.int64, torch.int32) or idx.dim() != 2:
+        raise ValueError("idx must be a 2-D int64 or int32 tensor")
+    T, k = idx.shape
+    if out is None:
+        out = empty_layout(T, k, E, R, idx.device)
+    _check(lib().ep_get_layout_noalloc(
+        _ptr(idx), int(idx.dtype == torch.int64), T, k, E, R,
+        _ptr(out.cnt_e), _ptr(out.cnt_r), _ptr(out.in_rank), _ptr(out.off_e),
+        _ptr(out.off_r), _ptr(out.slot_pos), _ptr(out.recv_src),
         _ptr(d_err), _stream(stream)))
     return out
 

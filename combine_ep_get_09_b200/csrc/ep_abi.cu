@@ -63,6 +63,14 @@ ep_status_t check_rows(const char *fn, int T, int H, int k, int num_sms) {
 
 namespace ep {
 
+ep_status_t record_error(ep_status_t status, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return status;
+}
+
 int device_sm_count() {
   static int cached[64] = {};
   int dev = 0;
@@ -236,3 +244,33 @@ ep_status_t ep_read_error(const int32_t *d_err, void *stream) {
 }
 
 }  // extern "C"
+
+namespace ep {
+
+// The argument checks of ep_get_layout minus the workspace, for entry
+// points that supply their own scratch.
+ep_status_t check_layout_args(const char *fn, const void *idx, int idx_is_int64, int T,
+                              int k, int E, int R, const int32_t *cnt_e,
+                              const int32_t *cnt_r, const uint8_t *in_rank,
+                              const int32_t *off_e, const int32_t *off_r,
+                              const int32_t *slot_pos, const int32_t *recv_src,
+                              const int32_t *d_err) {
+  g_err[0] = '\0';
+  ep_status_t st = check_layout_sizes(fn, T, k, E, R);
+  if (st != EP_OK) return st;
+  EP_REQUIRE_PTR(fn, cnt_e, 4);
+  EP_REQUIRE_PTR(fn, cnt_r, 4);
+  EP_REQUIRE_PTR(fn, off_e, 4);
+  EP_REQUIRE_PTR(fn, off_r, 4);
+  if (T > 0) {
+    EP_REQUIRE_PTR(fn, idx, idx_is_int64 ? 8 : 4);
+    EP_REQUIRE_PTR(fn, in_rank, 1);
+    EP_REQUIRE_PTR(fn, slot_pos, 4);
+    EP_REQUIRE_PTR(fn, recv_src, 4);
+  }
+  if (d_err != nullptr && !aligned(d_err, 4))
+    return fail(EP_ERR_INVALID_ARG, "%s: d_err is not 4-byte aligned", fn);
+  return EP_OK;
+}
+
+}  // namespace ep

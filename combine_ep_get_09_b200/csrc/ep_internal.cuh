@@ -76,6 +76,18 @@ cudaError_t launch_combine(const void *y, int T, int H, int k,
                            const int32_t *slot_pos, const float *w, void *out,
                            int num_sms, cudaStream_t s, int *launches);
 
+// Sets the message ep_last_error_string() returns on this host thread and
+// returns `status` (for entry points defined outside ep_abi.cu).
+ep_status_t record_error(ep_status_t status, const char *fmt, ...);
+
+// The argument checks ep_get_layout makes, except those of the workspace.
+ep_status_t check_layout_args(const char *fn, const void *idx, int idx_is_int64, int T,
+                              int k, int E, int R, const int32_t *cnt_e,
+                              const int32_t *cnt_r, const uint8_t *in_rank,
+                              const int32_t *off_e, const int32_t *off_r,
+                              const int32_t *slot_pos, const int32_t *recv_src,
+                              const int32_t *d_err);
+
 // SM count of the current device (cached per device).
 int device_sm_count();
 

@@ -158,6 +158,50 @@ ep_status_t ep_combine(const void *y, int T, int H, int k,
                        const int32_t *slot_pos, const float *w, void *out,
                        int num_sms, void *stream);
 
+/* Size of the scratch array behind ep_get_layout_noalloc (256 KiB). */
+#define EP_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+
+/*
+ * ep_get_layout_noalloc -- ep_get_layout for callers that cannot allocate
+ * device memory.
+ *
+ * The DeepEP pages have no counterpart to this entry point; it exists for
+ * deployments, not for the method.  Some callers cannot call cudaMalloc
+ * or keep a workspace of their own: a runtime whose device memory is all
+ * handed out up front by its own pool (an extra allocation would fail or
+ * break its accounting), or a latency-critical loop that must not pay the
+ * implicit device-wide synchronisation of cudaMalloc / cudaFree.  This
+ * variant takes the same arguments as ep_get_layout minus ws / ws_bytes
+ * and computes the same outputs.  Its scratch is a fixed array of
+ * EP_NOALLOC_SCRATCH_BYTES bytes inside the library: every GPU that loads
+ * the library holds one copy of it until the process exits, and the call
+ * itself allocates nothing (no cudaMalloc, no cudaFree, no allocating
+ * library routine).
+ *
+ * Limits: a batch whose tiled layout needs more scratch than the array
+ * (ep_layout_workspace_bytes(T, k, E, R) > EP_NOALLOC_SCRATCH_BYTES, e.g.
+ * very large T with E near EP_MAX_E) is rejected with EP_ERR_UNSUPPORTED
+ * and a message, before anything is enqueued.  The prefill, skewed and
+ * large workloads (up to 32768 tokens, 256 experts) all fit.
+ *
+ * Set-up: the first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture begins.
+ *
+ * Sharing: every call on a device uses the same array, which keeps the
+ * last call's contents; each call clears the part that must start at
+ * zero (the 16-byte ticket) on `stream` before its kernels run.  Calls
+ * whose work overlaps on the GPU (different streams, no ordering between
+ * them) race on the array and give wrong layouts: order them on one
+ * stream, or use ep_get_layout with one workspace per stream.
+ */
+ep_status_t ep_get_layout_noalloc(const void *idx, int idx_is_int64, int T,
+                                  int k, int E, int R, int32_t *cnt_e,
+                                  int32_t *cnt_r, uint8_t *in_rank,
+                                  int32_t *off_e, int32_t *off_r,
+                                  int32_t *slot_pos, int32_t *recv_src,
+                                  int32_t *d_err, void *stream);
+
 /*
  * Waits for `stream` and returns the device error word *d_err (EP_OK when
  * no bad id was met), or EP_ERR_CUDA if the copy failed.
