@@ -7,8 +7,10 @@ One step = one pass of the whole path over one batch of the 4096-token
 prefill workload (hidden 7168, 256 experts in 8 logical ranks, top-8,
 group-limited routing): dispatch layout, bf16 dispatch, FP8 dispatch, and
 the gate-weighted combine of the bf16 receive buffer (identity experts).
-Inputs are resident in HBM when the timed region starts; L2 is flushed
-(256 MiB write) between steps, outside the per-step CUDA events.
+Inputs are resident in HBM when the timed region starts.  Between steps the
+L2 is flushed outside the per-step CUDA events: a 256 MiB write evicts the
+step's data, then a 256 MiB read pushes the flush's own dirty lines back to
+HBM, so no step pays for write-backs that are not its own.
 
 Prints one JSON line.  ``value`` is algorithmic HBM bytes moved per second
 over all ranks (each source byte read once, each destination byte written
@@ -29,9 +31,7 @@ import json
 import os
 import re
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -47,6 +47,20 @@ METRIC = ("dispatch+combine HBM GB/s (% of B200 peak); "
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
 L2_FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Write a buffer larger than L2 (evicting everything), then read another
+    one so that the write's dirty lines are written back now rather than
+    during the next timed kernel."""
+
+    def __init__(self, device):
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
 
 
 # ------------------------------------------------------------- bytes model
@@ -82,65 +96,77 @@ def measured_peak():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
-              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons sampled through NVML every
+    2 ms in a background thread while the timed region runs (plus one sample
+    as it starts and one as it ends).  Read-only:
+    no clock or other GPU setting is touched."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
     def __init__(self, device):
-        # address the GPU by UUID: local CUDA indices may be remapped
+        self.device = device
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.error = None
+        self._stop = None
+        self._thread = None
+
+    def _handle(self, nv):
+        props = torch.cuda.get_device_properties(self.device)
         try:
-            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
-        except Exception:  # noqa: BLE001 - older torch without .uuid
-            self.dev = str(device.index)
-        self.proc = None
-        self.file = None
+            return nv.nvmlDeviceGetHandleByUUID(("GPU-" + str(props.uuid)).encode())
+        except Exception:  # noqa: BLE001 - fall back to the PCI address
+            bus = (f"{getattr(props, 'pci_domain_id', 0):08x}:{props.pci_bus_id:02x}:"
+                   f"{props.pci_device_id:02x}.0")
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
 
     def __enter__(self):
+        import threading
         try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.dev), "-lms", "200"], stdout=self.file,
-                stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - no NVML: report no clocks
+            self.error = repr(e)
+            return self
+        self._stop = threading.Event()
+
+        def sample():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, attr in self.REASONS:
+                    if mask & getattr(nv, attr):
+                        self.reasons.add(name)
+                return True
+            except Exception as e:  # noqa: BLE001
+                self.error = repr(e)
+                return False
+
+        def run():
+            while not self._stop.is_set() and sample():
+                self._stop.wait(0.002)
+            sample()
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or self.file is None:
-            return None
-        self.file.flush()
-        with open(self.file.name) as f:
-            rows = [r.strip().split(", ") for r in f if r.strip()]
-        os.unlink(self.file.name)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            if len(r) < 9:
-                continue
-            try:
-                sm.append(float(r[1]))
-                mx = float(r[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, r[5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "error": self.error}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 def dist_env():
@@ -204,14 +230,16 @@ class Step:
         if events is not None:
             events[1].record(stream)
         if not fp8_only:
-            ep.ep_dispatch(self.x, self.layout.slot_pos, recv=self.recv, stream=stream)
+            ep.ep_dispatch(self.x, self.layout.slot_pos, recv=self.recv,
+                           d_err=self.d_err, stream=stream)
         if events is not None:
             events[2].record(stream)
         ep.ep_dispatch(self.x, self.layout.slot_pos, fp8=True, recv=self.recv_q,
-                       recv_scale=self.recv_s, stream=stream)
+                       recv_scale=self.recv_s, d_err=self.d_err, stream=stream)
         if events is not None:
             events[3].record(stream)
-        ep.ep_combine(self.recv, self.layout.slot_pos, self.w, out=self.out, stream=stream)
+        ep.ep_combine(self.recv, self.layout.slot_pos, self.w, out=self.out,
+                      d_err=self.d_err, stream=stream)
         if events is not None:
             events[4].record(stream)
 
@@ -226,17 +254,17 @@ def bench_ours(args, world, rank, device):
     batch = workloads.make_batch(cfg, seed=rank)
     st = Step(ep, cfg, batch, device)
     stream = torch.cuda.Stream(device)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     nbytes = step_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R)
     total_bytes = sum(nbytes.values())
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            flush.zero_()
+            flush()
             st.run(stream)
     stream.synchronize()
     if ep.ep_read_error(st.d_err, stream) != 0:
-        raise RuntimeError("device reported a bad expert id")
+        raise RuntimeError("the device reported an error during warm-up")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     barrier(world)
@@ -244,12 +272,14 @@ def bench_ours(args, world, rank, device):
     launches0 = ep.ep_kernel_launches()
     with ClockSampler(device) as clocks, torch.cuda.stream(stream):
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             st.run(stream, evs[i])
         stream.synchronize()
     torch.cuda.synchronize(device)
     barrier(world)
     launches = ep.ep_kernel_launches() - launches0
+    if ep.ep_read_error(st.d_err, stream) != 0:
+        raise RuntimeError("the device reported an error in the timed steps")
 
     per_kernel = {n: [] for n in KERNELS}
     step_ms = []
@@ -291,7 +321,8 @@ def bench_ours(args, world, rank, device):
                          "layout + bf16 dispatch + FP8 dispatch + combine"),
             "T": cfg.T, "H": cfg.H, "E": cfg.E, "R": cfg.R, "k": cfg.k,
             "bytes_per_step": total_bytes,
-            "l2": "flushed between steps (256 MiB write), outside the step events",
+            "l2": ("flushed between steps outside the step events: 256 MiB write, "
+                   "then 256 MiB read"),
             "parallelism": f"{world} independent batch(es), one per GPU",
         },
         "frac_of_8TBs": round(value / world / SPEC_HBM_GBS, 4),
@@ -384,7 +415,7 @@ def bench_e2e(ep, cfg, batch, device, args, world, total_bytes):
     h_out = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
     st = Step(ep, cfg, batch, device)
     stream = torch.cuda.Stream(device)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
 
     def one(evs=None):
         if evs is not None:
@@ -399,7 +430,7 @@ def bench_e2e(ep, cfg, batch, device, args, world, total_bytes):
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
-            flush.zero_()
+            flush()
             one()
     stream.synchronize()
     n = max(3, min(args.steps, 10))
@@ -407,7 +438,7 @@ def bench_e2e(ep, cfg, batch, device, args, world, total_bytes):
     barrier(world)
     with torch.cuda.stream(stream):
         for i in range(n):
-            flush.zero_()
+            flush()
             one(evs[i])
     stream.synchronize()
     barrier(world)
@@ -491,7 +522,7 @@ def bench_reference(args, world, rank):
 def main():
     p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--skip-decode", action="store_true")

@@ -24,13 +24,14 @@ __all__ = ["EPError", "EPLibraryError", "Layout", "ep_get_layout",
            "ep_dispatch", "ep_combine", "ep_read_error",
            "ep_layout_workspace_bytes", "ep_kernel_launches", "lib",
            "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_UNSUPPORTED", "EP_ERR_CUDA",
-           "EP_ERR_INDEX", "LIB_PATH"]
+           "EP_ERR_INDEX", "EP_ERR_TIMEOUT", "LIB_PATH"]
 
 EP_OK = 0
 EP_ERR_INVALID_ARG = 1
 EP_ERR_UNSUPPORTED = 2
 EP_ERR_CUDA = 3
 EP_ERR_INDEX = 4
+EP_ERR_TIMEOUT = 5
 EP_NOALLOC_SCRATCH_BYTES = 256 * 1024
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep.so")
@@ -59,8 +60,8 @@ _SIGNATURES = {
     "ep_layout_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "ep_get_layout": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                        _vp, _vp, _sz, _vp, _vp], _i),
-    "ep_dispatch": ([_vp, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp], _i),
-    "ep_combine": ([_vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp], _i),
+    "ep_dispatch": ([_vp, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp], _i),
+    "ep_combine": ([_vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp], _i),
     "ep_read_error": ([_vp, _vp], _i),
     "ep_get_layout_noalloc": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                _vp, _vp, _vp, _vp], _i),
@@ -187,7 +188,8 @@ def ep_get_layout_noalloc(idx: torch.Tensor, E: int, R: int, *,
 def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
                 recv: Optional[torch.Tensor] = None,
                 recv_scale: Optional[torch.Tensor] = None,
-                num_sms: int = 0, stream=None):
+                num_sms: int = 0, d_err: Optional[torch.Tensor] = None,
+                stream=None):
     """Rows of ``x`` [T, H] bf16 to their receive rows.  Returns ``recv``
     [T*k, H] (bf16), or ``(recv_q [T*k, H] float8_e4m3fn, recv_scale
     [T*k, H/128] fp32)`` when ``fp8``."""
@@ -205,12 +207,13 @@ def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
                                  dtype=torch.float32)
     _check(lib().ep_dispatch(_ptr(x), T, H, k, _ptr(slot_pos), int(bool(fp8)),
                              _ptr(recv), _ptr(recv_scale) if fp8 else None,
-                             num_sms, _stream(stream)))
+                             num_sms, _ptr(d_err), _stream(stream)))
     return (recv, recv_scale) if fp8 else recv
 
 
 def ep_combine(y: torch.Tensor, slot_pos: torch.Tensor, w: torch.Tensor, *,
                out: Optional[torch.Tensor] = None, num_sms: int = 0,
+               d_err: Optional[torch.Tensor] = None,
                stream=None) -> torch.Tensor:
     """Gate-weighted combine of expert outputs ``y`` [T*k, H] bf16 into
     ``out`` [T, H] bf16 (fp32 fma chain in slot order)."""
@@ -225,7 +228,7 @@ def ep_combine(y: torch.Tensor, slot_pos: torch.Tensor, w: torch.Tensor, *,
     if out is None:
         out = torch.empty((T, H), device=y.device, dtype=torch.bfloat16)
     _check(lib().ep_combine(_ptr(y), T, H, k, _ptr(slot_pos), _ptr(w),
-                            _ptr(out), num_sms, _stream(stream)))
+                            _ptr(out), num_sms, _ptr(d_err), _stream(stream)))
     return out
 
 

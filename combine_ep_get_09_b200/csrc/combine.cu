@@ -1,21 +1,33 @@
 // combine.cu -- gate-weighted sum of the expert outputs back into token
 // order: out[t] = bf16(fma chain over slots j = 0..k-1 of w[t,j] * y[row]).
 //
-// Persistent grid-stride loop over work items (token t, chunk of its row).
-// For each item a warp issues the loads of up to 8 slot rows at once
-// (128-bit read-only streaming loads, so 8 x 16 B per lane are in flight),
-// then folds them into fp32 accumulators strictly in slot order, and writes
-// the chunk once with a coalesced streaming store.
+// Two kernels, both fp32 fma chains in slot order (so both bit-identical):
+//
+//  * combine_bulk_kernel (k <= 8, the common case): a bulk-copy (TMA)
+//    pipeline.  A CTA of kChunkVec threads walks a contiguous range of
+//    work items (token t, chunk c of kChunkVec 16-byte vectors).  Thread 0
+//    gathers the chunk of each of the token's k slot rows into shared
+//    memory with cp.async.bulk (one copy per row, completing on the stage's
+//    mbarrier), kStages items ahead; every thread then folds its 16 bytes
+//    of the k rows and writes one 16-byte vector of the output.  The bytes
+//    in flight live in shared memory, not registers, which is what keeps
+//    HBM busy on this read-dominated gather.
+//  * combine_reg_kernel (any k <= 32): a warp per item with 128-bit loads
+//    of 8 slot rows at a time into registers.
 #include <cuda_bf16.h>
 
+#include "bulk.cuh"
 #include "ep_internal.cuh"
 
 namespace ep {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kVec = 1;      // 16-byte vectors per lane per item
-constexpr int kSlotBatch = 8;  // slot rows loaded together
+constexpr int kRegThreads = 256;
+constexpr int kSlotBatch = 8;    // slot rows loaded together (register path)
+constexpr int kBulkMaxK = 8;     // slot rows one bulk stage holds
+constexpr int kChunkVec = 256;   // 16-byte vectors per row chunk = threads
+constexpr int kStages = 2;       // items in flight per CTA
+constexpr int kBulkSmem = kStages * kBulkMaxK * kChunkVec * 16;
 
 __device__ __forceinline__ void fma_bf16x8(float *acc, float w, uint4 v) {
   const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -36,15 +48,101 @@ __device__ __forceinline__ uint4 to_bf16x8(const float *acc) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <int V>
-__global__ void __launch_bounds__(kThreads, 2)
-    combine_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
-                   const int32_t *__restrict__ slot_pos,
-                   const float *__restrict__ w, uint4 *__restrict__ out,
-                   long n_rows) {
+__global__ void __launch_bounds__(kChunkVec)
+    combine_bulk_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
+                        const int32_t *__restrict__ slot_pos, const float *__restrict__ w,
+                        uint4 *__restrict__ out, long n_rows, int32_t *d_err) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  uint4 *stage_buf = reinterpret_cast<uint4 *>(smem_raw);  // [kStages][kBulkMaxK][kChunkVec]
+  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ int stage_row[kStages][kBulkMaxK];
+  __shared__ float stage_w[kStages][kBulkMaxK];
+  __shared__ int timed_out;
+
+  const int tid = threadIdx.x;
+  const int nchunks = (Hv + kChunkVec - 1) / kChunkVec;
+  const long items = static_cast<long>(T) * nchunks;
+  const long per_cta = (items + gridDim.x - 1) / gridDim.x;
+  const long first = min(items, static_cast<long>(blockIdx.x) * per_cta);
+  const long n_mine = min(items, first + per_cta) - first;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    mbar_init_fence();
+    timed_out = 0;
+  }
+  __syncthreads();
+
+  // thread 0: gather item i's slot rows into stage i % kStages
+  auto issue = [&](long i) {
+    const long it = first + i;
+    const int s = static_cast<int>(i % kStages);
+    const int t = static_cast<int>(it / nchunks);
+    const int v0 = static_cast<int>(it % nchunks) * kChunkVec;
+    const unsigned bytes = static_cast<unsigned>(min(kChunkVec, Hv - v0)) * 16u;
+    int rows[kBulkMaxK];
+    int n_valid = 0;
+#pragma unroll
+    for (int j = 0; j < kBulkMaxK; ++j) {
+      int r = -1;
+      float wj = 0.0f;
+      if (j < k) {
+        r = __ldg(slot_pos + static_cast<long>(t) * k + j);
+        wj = __ldg(w + static_cast<long>(t) * k + j);
+        if (r < 0 || r >= n_rows) r = -1;
+      }
+      rows[j] = r;
+      stage_row[s][j] = r;
+      stage_w[s][j] = wj;
+      n_valid += r >= 0;
+    }
+    // the arrival publishes stage_row / stage_w (release) with the byte count
+    mbar_arrive_expect_tx(&full[s], n_valid * bytes);
+#pragma unroll
+    for (int j = 0; j < kBulkMaxK; ++j)
+      if (rows[j] >= 0)
+        bulk_load(stage_buf + (s * kBulkMaxK + j) * kChunkVec,
+                  y + static_cast<long>(rows[j]) * Hv + v0, bytes, &full[s]);
+  };
+
+  if (tid == 0)
+    for (long i = 0; i < min(static_cast<long>(kStages), n_mine); ++i) issue(i);
+
+  long i = 0;
+  for (; i < n_mine; ++i) {
+    const int s = static_cast<int>(i % kStages);
+    const long it = first + i;
+    const int t = static_cast<int>(it / nchunks);
+    const int v0 = static_cast<int>(it % nchunks) * kChunkVec;
+    if (!mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1))) timed_out = 1;
+    if (tid < Hv - v0) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < kBulkMaxK; ++j)
+        if (stage_row[s][j] >= 0)  // dropped slots add nothing
+          fma_bf16x8(acc, stage_w[s][j], stage_buf[(s * kBulkMaxK + j) * kChunkVec + tid]);
+      st_stream_v4(out + static_cast<long>(t) * Hv + v0 + tid, to_bf16x8(acc));
+    }
+    __syncthreads();  // stage s fully read
+    if (timed_out) break;
+    if (tid == 0 && i + kStages < n_mine) issue(i + kStages);
+  }
+  if (timed_out && tid == 0) {
+    if (d_err != nullptr) atomicExch(reinterpret_cast<int *>(d_err), EP_ERR_TIMEOUT);
+    // let the copies still in flight land before the CTA's memory goes away
+    for (long q = i + 1; q < min(n_mine, i + kStages); ++q)
+      mbar_wait_bounded(&full[q % kStages], static_cast<unsigned>((q / kStages) & 1));
+  }
+}
+
+__global__ void __launch_bounds__(kRegThreads, 2)
+    combine_reg_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
+                       const int32_t *__restrict__ slot_pos, const float *__restrict__ w,
+                       uint4 *__restrict__ out, long n_rows) {
   const int lane = threadIdx.x & 31;
-  const int per_chunk = 32 * V;
-  const int nchunks = (Hv + per_chunk - 1) / per_chunk;
+  const int nchunks = (Hv + 31) / 32;
   const long items = static_cast<long>(T) * nchunks;
   const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
   for (long it = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -54,16 +152,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     const long tk = static_cast<long>(t) * k;
     const int sp = lane < k ? __ldg(slot_pos + tk + lane) : -1;
     const float wt = lane < k ? __ldg(w + tk + lane) : 0.0f;
-    const int v0 = c * per_chunk + lane;
+    const int v = c * 32 + lane;
 
-    float acc[V][8];
+    float acc[8];
 #pragma unroll
-    for (int u = 0; u < V; ++u)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[u][e] = 0.0f;
-
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
     for (int j0 = 0; j0 < k; j0 += kSlotBatch) {
-      uint4 v[kSlotBatch][V];
+      uint4 val[kSlotBatch];
       float wj[kSlotBatch];
       bool ok[kSlotBatch];
 #pragma unroll
@@ -72,39 +167,46 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int row = __shfl_sync(0xffffffffu, sp, j & 31);
         wj[jj] = __shfl_sync(0xffffffffu, wt, j & 31);
         ok[jj] = j < k && row >= 0 && row < n_rows;
-        const uint4 *src = y + static_cast<long>(row) * Hv;
-#pragma unroll
-        for (int u = 0; u < V; ++u)
-          v[jj][u] = ok[jj] && v0 + 32 * u < Hv ? ld_stream_v4(src + v0 + 32 * u)
-                                                : make_uint4(0, 0, 0, 0);
+        val[jj] = ok[jj] && v < Hv ? ld_stream_v4(y + static_cast<long>(row) * Hv + v)
+                                   : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int jj = 0; jj < kSlotBatch; ++jj) {
-        if (!ok[jj]) continue;  // a dropped slot adds nothing
-#pragma unroll
-        for (int u = 0; u < V; ++u) fma_bf16x8(acc[u], wj[jj], v[jj][u]);
-      }
+      for (int jj = 0; jj < kSlotBatch; ++jj)
+        if (ok[jj]) fma_bf16x8(acc, wj[jj], val[jj]);  // dropped slots add nothing
     }
-    uint4 *dst = out + static_cast<long>(t) * Hv;
-#pragma unroll
-    for (int u = 0; u < V; ++u)
-      if (v0 + 32 * u < Hv) st_stream_v4(dst + v0 + 32 * u, to_bf16x8(acc[u]));
+    if (v < Hv) st_stream_v4(out + static_cast<long>(t) * Hv + v, to_bf16x8(acc));
   }
 }
 
 }  // namespace
 
-cudaError_t launch_combine(const void *y, int T, int H, int k,
-                           const int32_t *slot_pos, const float *w, void *out,
-                           int num_sms, cudaStream_t s, int *launches) {
+cudaError_t launch_combine(const void *y, int T, int H, int k, const int32_t *slot_pos,
+                           const float *w, void *out, int num_sms, int32_t *d_err,
+                           cudaStream_t s, int *launches) {
   const int Hv = H / 8;
-  const long nchunks = (Hv + 32 * kVec - 1) / (32 * kVec);
-  const long items = static_cast<long>(T) * nchunks;
+  const long n_rows = static_cast<long>(T) * k;
+  if (k <= kBulkMaxK) {
+    const long items = static_cast<long>(T) * ((Hv + kChunkVec - 1) / kChunkVec);
+    if (items == 0) return cudaSuccess;
+    const cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(combine_bulk_kernel),
+                                               kBulkSmem);
+    if (err != cudaSuccess) return err;
+    // CTAs: one per item, capped at the CTAs that fit on the SMs at once
+    const long grid = persistent_grid(reinterpret_cast<const void *>(combine_bulk_kernel),
+                                      kChunkVec, kBulkSmem, items * (kChunkVec / kWarp),
+                                      num_sms);
+    combine_bulk_kernel<<<grid, kChunkVec, kBulkSmem, s>>>(
+        static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w, static_cast<uint4 *>(out), n_rows,
+        d_err);
+    ++*launches;
+    return cudaGetLastError();
+  }
+  const long items = static_cast<long>(T) * ((Hv + 31) / 32);
   if (items == 0) return cudaSuccess;
-  auto kern = combine_kernel<kVec>;
-  const long grid = persistent_grid(reinterpret_cast<const void *>(kern), kThreads, items, num_sms);
-  kern<<<grid, kThreads, 0, s>>>(static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,
-                                 static_cast<uint4 *>(out), static_cast<long>(T) * k);
+  const long grid = persistent_grid(reinterpret_cast<const void *>(combine_reg_kernel),
+                                    kRegThreads, 0, items, num_sms);
+  combine_reg_kernel<<<grid, kRegThreads, 0, s>>>(static_cast<const uint4 *>(y), T, Hv, k,
+                                                  slot_pos, w, static_cast<uint4 *>(out), n_rows);
   ++*launches;
   return cudaGetLastError();
 }

@@ -146,13 +146,15 @@ __global__ void __launch_bounds__(kThreads)
 
 cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
                                  const int32_t *slot_pos, void *recv,
-                                 int num_sms, cudaStream_t s, int *launches) {
+                                 int num_sms, int32_t * /*d_err*/, cudaStream_t s,
+                                 int *launches) {
   const int Hv = H / 8;
   const long nchunks = (Hv + 32 * kBf16Vec - 1) / (32 * kBf16Vec);
   const long items = static_cast<long>(T) * nchunks;
   if (items == 0) return cudaSuccess;
   auto kern = dispatch_bf16_kernel<kBf16Vec>;
-  const long grid = persistent_grid(reinterpret_cast<const void *>(kern), kThreads, items, num_sms);
+  const long grid =
+      persistent_grid(reinterpret_cast<const void *>(kern), kThreads, 0, items, num_sms);
   kern<<<grid, kThreads, 0, s>>>(static_cast<const uint4 *>(x), T, Hv, k, slot_pos,
                                  static_cast<uint4 *>(recv), static_cast<long>(T) * k);
   ++*launches;
@@ -161,13 +163,13 @@ cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
 
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
-                                float *recv_scale, int num_sms,
+                                float *recv_scale, int num_sms, int32_t * /*d_err*/,
                                 cudaStream_t s, int *launches) {
   const long nchunks = (H / 128 + 3) / 4;
   const long items = static_cast<long>(T) * nchunks;
   if (items == 0) return cudaSuccess;
   const long grid = persistent_grid(reinterpret_cast<const void *>(dispatch_fp8_kernel),
-                                    kThreads, items, num_sms);
+                                    kThreads, 0, items, num_sms);
   dispatch_fp8_kernel<<<grid, kThreads, 0, s>>>(
       static_cast<const uint4 *>(x), T, H, k, slot_pos, static_cast<uint2 *>(recv_q),
       recv_scale, static_cast<long>(T) * k);

@@ -83,7 +83,8 @@ int device_sm_count() {
   return n;
 }
 
-long persistent_grid(const void *kernel, int threads, long items, int num_sms) {
+long persistent_grid(const void *kernel, int threads, int smem_bytes, long warp_items,
+                     int num_sms) {
   static std::mutex mu;
   static std::map<std::pair<int, const void *>, int> cache;
   int dev = 0;
@@ -95,7 +96,7 @@ long persistent_grid(const void *kernel, int threads, long items, int num_sms) {
     if (it != cache.end()) {
       per_sm = it->second;
     } else {
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) !=
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem_bytes) !=
               cudaSuccess ||
           per_sm < 1)
         per_sm = 1;
@@ -104,16 +105,30 @@ long persistent_grid(const void *kernel, int threads, long items, int num_sms) {
   }
   const int sms = num_sms > 0 ? num_sms : device_sm_count();
   const long warps_per_block = threads / kWarp;
-  const long need = (items + warps_per_block - 1) / warps_per_block;
+  const long need = (warp_items + warps_per_block - 1) / warps_per_block;
   const long cap = static_cast<long>(sms) * per_sm;
   return need < cap ? need : cap;
+}
+
+cudaError_t raise_dynamic_smem(const void *kernel, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void *>, int> done;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({dev, kernel});
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess) done[{dev, kernel}] = bytes;
+  return err;
 }
 
 }  // namespace ep
 
 extern "C" {
 
-int ep_abi_version(void) { return 1; }
+int ep_abi_version(void) { return 2; }
 
 const char *ep_last_error_string(void) { return g_err; }
 
@@ -191,7 +206,7 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
 
 ep_status_t ep_dispatch(const void *x, int T, int H, int k,
                         const int32_t *slot_pos, int fp8, void *recv,
-                        float *recv_scale, int num_sms, void *stream) {
+                        float *recv_scale, int num_sms, int32_t *d_err, void *stream) {
   static const char fn[] = "ep_dispatch";
   g_err[0] = '\0';
   ep_status_t st = check_rows(fn, T, H, k, num_sms);
@@ -203,18 +218,20 @@ ep_status_t ep_dispatch(const void *x, int T, int H, int k,
   EP_REQUIRE_PTR(fn, slot_pos, 4);
   EP_REQUIRE_PTR(fn, recv, 16);
   if (fp8) EP_REQUIRE_PTR(fn, recv_scale, 4);
+  if (d_err != nullptr && !aligned(d_err, 4))
+    return fail(EP_ERR_INVALID_ARG, "%s: d_err is not 4-byte aligned", fn);
   int n = 0;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
-      fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale, num_sms, s, &n)
-          : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, num_sms, s, &n);
+      fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale, num_sms, d_err, s, &n)
+          : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, num_sms, d_err, s, &n);
   g_launches += n;
   return from_cuda(e, fn);
 }
 
 ep_status_t ep_combine(const void *y, int T, int H, int k,
                        const int32_t *slot_pos, const float *w, void *out,
-                       int num_sms, void *stream) {
+                       int num_sms, int32_t *d_err, void *stream) {
   static const char fn[] = "ep_combine";
   g_err[0] = '\0';
   ep_status_t st = check_rows(fn, T, H, k, num_sms);
@@ -224,8 +241,10 @@ ep_status_t ep_combine(const void *y, int T, int H, int k,
   EP_REQUIRE_PTR(fn, slot_pos, 4);
   EP_REQUIRE_PTR(fn, w, 4);
   EP_REQUIRE_PTR(fn, out, 16);
+  if (d_err != nullptr && !aligned(d_err, 4))
+    return fail(EP_ERR_INVALID_ARG, "%s: d_err is not 4-byte aligned", fn);
   int n = 0;
-  const cudaError_t e = ep::launch_combine(y, T, H, k, slot_pos, w, out, num_sms,
+  const cudaError_t e = ep::launch_combine(y, T, H, k, slot_pos, w, out, num_sms, d_err,
                                            static_cast<cudaStream_t>(stream), &n);
   g_launches += n;
   return from_cuda(e, fn);

@@ -67,14 +67,16 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s, int *launches);
 
 cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
                                  const int32_t *slot_pos, void *recv,
-                                 int num_sms, cudaStream_t s, int *launches);
+                                 int num_sms, int32_t *d_err, cudaStream_t s,
+                                 int *launches);
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
-                                float *recv_scale, int num_sms,
+                                float *recv_scale, int num_sms, int32_t *d_err,
                                 cudaStream_t s, int *launches);
 cudaError_t launch_combine(const void *y, int T, int H, int k,
                            const int32_t *slot_pos, const float *w, void *out,
-                           int num_sms, cudaStream_t s, int *launches);
+                           int num_sms, int32_t *d_err, cudaStream_t s,
+                           int *launches);
 
 // Sets the message ep_last_error_string() returns on this host thread and
 // returns `status` (for entry points defined outside ep_abi.cu).
@@ -91,10 +93,15 @@ ep_status_t check_layout_args(const char *fn, const void *idx, int idx_is_int64,
 // SM count of the current device (cached per device).
 int device_sm_count();
 
-// Grid for a persistent grid-stride kernel: enough blocks of `threads`
-// threads (warps_per_item = 1) to cover `items` warp work items, capped at
-// the blocks that fit at once on `num_sms` SMs (0 = all SMs).  The
-// occupancy figure is cached per (device, kernel).
-long persistent_grid(const void *kernel, int threads, long items, int num_sms);
+// Grid for a persistent kernel: enough blocks of `threads` threads to give
+// each of `warp_items` work items a warp, capped at the blocks that fit at
+// once (with `smem_bytes` of dynamic shared memory each) on `num_sms` SMs
+// (0 = all SMs).  The occupancy figure is cached per (device, kernel).
+long persistent_grid(const void *kernel, int threads, int smem_bytes, long warp_items,
+                     int num_sms);
+
+// Raises a kernel's dynamic shared memory limit to `bytes` (once per
+// device and kernel).
+cudaError_t raise_dynamic_smem(const void *kernel, int bytes);
 
 }  // namespace ep

@@ -26,9 +26,12 @@
  *    device memory.
  *  - Argument errors are returned before anything is enqueued; nothing is
  *    written then.  EP_ERR_CUDA means a launch failed; the message is in
- *    ep_last_error_string().  Nothing ever traps on the device: a bad
- *    expert id found on the device is written to *d_err (EP_ERR_INDEX) and
- *    its slot is treated as dropped.
+ *    ep_last_error_string().  Nothing ever traps on the device: problems
+ *    found on the device are written to the caller's optional error word
+ *    d_err (device int32, may be NULL; never cleared by the library) --
+ *    EP_ERR_INDEX for a bad expert id (its slot is treated as dropped),
+ *    EP_ERR_TIMEOUT if a kernel's bounded wait for its own asynchronous
+ *    copies gave up (it then stops early instead of hanging).
  *  - Pointers must be 16-byte aligned unless stated otherwise.
  */
 #ifndef EP_H_
@@ -48,12 +51,14 @@ typedef int ep_status_t;
 #define EP_ERR_UNSUPPORTED 2 /* valid request outside the built limits   */
 #define EP_ERR_CUDA 3        /* a CUDA call failed; see ep_last_error_string */
 #define EP_ERR_INDEX 4       /* device-side: an expert id outside [-1, E) */
+#define EP_ERR_TIMEOUT 5     /* device-side: a bounded wait for an async copy
+                                gave up; that call's output is incomplete */
 
 #define EP_MAX_K 32    /* top-k slots per token            */
 #define EP_MAX_E 1024  /* experts                          */
 #define EP_MAX_R 64    /* logical ranks                    */
 
-/* Version of this ABI (incremented on any signature change). */
+/* Version of this ABI (incremented on any signature change): 2. */
 int ep_abi_version(void);
 
 /* Message of the last error returned on this host thread ("" if none). */
@@ -134,10 +139,12 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
  * T >= 0, 1 <= k <= EP_MAX_K, H > 0 with H % 8 == 0 (H % 128 == 0 for
  * fp8), T*k < 2^31.
  * num_sms     SMs to spread the work over (0 = all of them).
+ * d_err       optional device error word (see the conventions above).
  */
 ep_status_t ep_dispatch(const void *x, int T, int H, int k,
                         const int32_t *slot_pos, int fp8, void *recv,
-                        float *recv_scale, int num_sms, void *stream);
+                        float *recv_scale, int num_sms, int32_t *d_err,
+                        void *stream);
 
 /*
  * ep_combine -- bring the expert outputs back to their tokens.
@@ -152,11 +159,11 @@ ep_status_t ep_dispatch(const void *x, int T, int H, int k,
  * slot_pos   [T,k] int32; values outside [0, T*k) are skipped.
  * w          [T,k] fp32 gate weights (4-byte aligned).
  * out        [T,H] bf16; a token with no kept slot gets +0.
- * Limits as ep_dispatch (H % 8 == 0).
+ * Limits as ep_dispatch (H % 8 == 0).  num_sms and d_err as ep_dispatch.
  */
 ep_status_t ep_combine(const void *y, int T, int H, int k,
                        const int32_t *slot_pos, const float *w, void *out,
-                       int num_sms, void *stream);
+                       int num_sms, int32_t *d_err, void *stream);
 
 /* Size of the scratch array behind ep_get_layout_noalloc (256 KiB). */
 #define EP_NOALLOC_SCRATCH_BYTES (256u * 1024u)
@@ -178,11 +185,13 @@ ep_status_t ep_combine(const void *y, int T, int H, int k,
  * itself allocates nothing (no cudaMalloc, no cudaFree, no allocating
  * library routine).
  *
- * Limits: a batch whose tiled layout needs more scratch than the array
+ * Limits: batches of up to 2^19 slots (T*k) use no scratch at all; a
+ * larger batch whose tiled layout needs more scratch than the array
  * (ep_layout_workspace_bytes(T, k, E, R) > EP_NOALLOC_SCRATCH_BYTES, e.g.
- * very large T with E near EP_MAX_E) is rejected with EP_ERR_UNSUPPORTED
- * and a message, before anything is enqueued.  The prefill, skewed and
- * large workloads (up to 32768 tokens, 256 experts) all fit.
+ * 100000 tokens, top-8 over 1024 experts) is rejected with
+ * EP_ERR_UNSUPPORTED and a message, before anything is enqueued.  For
+ * example 70000 tokens, top-8 over 128 experts in 16 ranks needs 170 KB
+ * and fits.
  *
  * Set-up: the first call on each device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current; make that

@@ -29,16 +29,20 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version():
-    assert ep.lib().ep_abi_version() == 1
+    assert ep.lib().ep_abi_version() == 2
 
 
 def test_workspace_sizes():
-    # single-block path needs none; the tiled path one row of E + R counts
-    # per tile plus a 16-byte ticket
+    # the cluster path (T*k <= 2^19) needs none; the tiled path one row of
+    # E + R counts per tile (at most 296 tiles of >= 128 tokens) plus a
+    # 16-byte ticket
     assert ep.ep_layout_workspace_bytes(128, 8, 256, 8) == 0
     assert ep.ep_layout_workspace_bytes(0, 8, 256, 8) == 0
-    assert ep.ep_layout_workspace_bytes(4096, 8, 256, 8) == 16 + 32 * 264 * 4
-    assert ep.ep_layout_workspace_bytes(32768, 8, 128, 16) == 16 + 256 * 144 * 4
+    assert ep.ep_layout_workspace_bytes(4096, 8, 256, 8) == 0
+    assert ep.ep_layout_workspace_bytes(65536, 8, 256, 8) == 0
+    assert ep.ep_layout_workspace_bytes(65537, 8, 256, 8) == 16 + 296 * 264 * 4
+    assert ep.ep_layout_workspace_bytes(70000, 8, 128, 16) == 16 + 296 * 144 * 4
+    assert ep.ep_layout_workspace_bytes(300000, 2, 16, 16) == 16 + 296 * 32 * 4
     # invalid sizes report 0
     assert ep.ep_layout_workspace_bytes(4096, 8, 250, 8) == 0
 
@@ -66,9 +70,9 @@ def _layout_call(**kw):
     (dict(idx=None), ep.EP_ERR_INVALID_ARG),
     (dict(idx=20), ep.EP_ERR_INVALID_ARG),       # int64 ids need 8-byte alignment
     (dict(slot_pos=18), ep.EP_ERR_INVALID_ARG),
-    (dict(T=4096, k=8, E=256, R=8), ep.EP_ERR_INVALID_ARG),   # tiled path, no ws
-    (dict(T=4096, k=8, E=256, R=8, ws=16, ws_bytes=100), ep.EP_ERR_INVALID_ARG),
-    (dict(T=4096, k=8, E=256, R=8, ws=24, ws_bytes=1 << 20), ep.EP_ERR_INVALID_ARG),
+    (dict(T=65537, k=8, E=256, R=8), ep.EP_ERR_INVALID_ARG),   # tiled path, no ws
+    (dict(T=65537, k=8, E=256, R=8, ws=16, ws_bytes=100), ep.EP_ERR_INVALID_ARG),
+    (dict(T=65537, k=8, E=256, R=8, ws=24, ws_bytes=1 << 20), ep.EP_ERR_INVALID_ARG),
 ])
 def test_layout_rejects(kw, status):
     assert _layout_call(**kw) == status
@@ -76,16 +80,17 @@ def test_layout_rejects(kw, status):
 
 
 @pytest.mark.parametrize("args,status", [
-    ((16, -1, 64, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
-    ((16, 4, 0, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
-    ((16, 4, 12, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_UNSUPPORTED),   # H % 8
-    ((16, 4, 64, 2, 16, 1, 16, 16, 0, None), ep.EP_ERR_UNSUPPORTED),     # fp8, H % 128
-    ((16, 4, 64, 33, 16, 0, 16, None, 0, None), ep.EP_ERR_UNSUPPORTED),  # k > 32
-    ((16, 4, 64, 2, 16, 0, 16, None, -1, None), ep.EP_ERR_INVALID_ARG),  # num_sms
-    ((None, 4, 64, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
-    ((24, 4, 64, 2, 16, 0, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),   # x misaligned
-    ((16, 4, 128, 2, 16, 1, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),  # fp8, no scale
-    ((16, 4, 64, 2, 16, 0, 8, None, 0, None), ep.EP_ERR_INVALID_ARG),    # recv misaligned
+    ((16, -1, 64, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 0, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 12, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_UNSUPPORTED),   # H % 8
+    ((16, 4, 64, 2, 16, 1, 16, 16, 0, None, None), ep.EP_ERR_UNSUPPORTED),     # fp8, H % 128
+    ((16, 4, 64, 33, 16, 0, 16, None, 0, None, None), ep.EP_ERR_UNSUPPORTED),  # k > 32
+    ((16, 4, 64, 2, 16, 0, 16, None, -1, None, None), ep.EP_ERR_INVALID_ARG),  # num_sms
+    ((None, 4, 64, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),
+    ((24, 4, 64, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),   # x misaligned
+    ((16, 4, 128, 2, 16, 1, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),  # fp8, no scale
+    ((16, 4, 64, 2, 16, 0, 8, None, 0, None, None), ep.EP_ERR_INVALID_ARG),    # recv misaligned
+    ((16, 4, 64, 2, 16, 0, 16, None, 0, 18, None), ep.EP_ERR_INVALID_ARG),     # d_err misaligned
 ])
 def test_dispatch_rejects(args, status):
     assert ep.lib().ep_dispatch(*args) == status
@@ -93,15 +98,16 @@ def test_dispatch_rejects(args, status):
 
 def test_dispatch_combine_empty_batch_is_a_no_op():
     # T = 0: valid, nothing to do, nothing touched (no device needed)
-    assert ep.lib().ep_dispatch(None, 0, 64, 2, None, 0, None, None, 0, None) == ep.EP_OK
-    assert ep.lib().ep_combine(None, 0, 64, 2, None, None, None, 0, None) == ep.EP_OK
+    assert ep.lib().ep_dispatch(None, 0, 64, 2, None, 0, None, None, 0, None, None) == ep.EP_OK
+    assert ep.lib().ep_combine(None, 0, 64, 2, None, None, None, 0, None, None) == ep.EP_OK
 
 
 @pytest.mark.parametrize("args,status", [
-    ((16, 4, 64, 2, 16, None, 16, 0, None), ep.EP_ERR_INVALID_ARG),  # no w
-    ((16, 4, 64, 2, 16, 18, 16, 0, None), ep.EP_ERR_INVALID_ARG),    # w misaligned
-    ((16, 4, 60, 2, 16, 16, 16, 0, None), ep.EP_ERR_UNSUPPORTED),
-    ((16, 4, 64, 2, 16, 16, 40, 0, None), ep.EP_ERR_INVALID_ARG),    # out misaligned
+    ((16, 4, 64, 2, 16, None, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),  # no w
+    ((16, 4, 64, 2, 16, 18, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),    # w misaligned
+    ((16, 4, 60, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_UNSUPPORTED),
+    ((16, 4, 64, 2, 16, 16, 40, 0, None, None), ep.EP_ERR_INVALID_ARG),    # out misaligned
+    ((16, 4, 64, 2, 16, 16, 16, 0, 2, None), ep.EP_ERR_INVALID_ARG),       # d_err misaligned
 ])
 def test_combine_rejects(args, status):
     assert ep.lib().ep_combine(*args) == status

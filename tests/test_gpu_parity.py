@@ -48,11 +48,13 @@ def test_layout_full_size(name, seed):
     assert_layout_equal(g, oracle.layout(b.idx, cfg.E, cfg.R))
 
 
-@pytest.mark.parametrize("T", [0, 1, 3, 31, 127, 2047, 2048, 2049, 4097, 9999])
+@pytest.mark.parametrize("T", [0, 1, 3, 31, 127, 512, 513, 2047, 4097, 9999, 32769,
+                               65536, 65537, 70001])
 @pytest.mark.parametrize("int32_ids", [False, True])
 def test_layout_ragged_and_both_id_types(T, int32_ids):
-    # T*k = 16384 (T = 2048, k = 8) is the largest single-block case;
-    # 2049 is the first tiled one
+    # k = 8: up to T = 512 one CTA, then a cluster of up to 16 CTAs (4096
+    # slots each, so 32769 is the first 16-CTA batch); T*k = 2^19
+    # (T = 65536) is the largest cluster case, 65537 the first tiled one
     cfg, b = _batch("prefill", 3, T=T, H=8, drop_frac=0.1, dup_frac=0.1)
     _, g = gpu_layout(b.idx, cfg.E, cfg.R, int32_ids=int32_ids)
     assert_layout_equal(g, oracle.layout(b.idx, cfg.E, cfg.R))
@@ -60,7 +62,8 @@ def test_layout_ragged_and_both_id_types(T, int32_ids):
 
 @pytest.mark.parametrize("T,k,E,R", [(500, 1, 1, 1), (300, 32, 64, 64),
                                      (2500, 32, 1024, 64), (4000, 4, 1024, 1),
-                                     (100000, 2, 16, 16)])
+                                     (100000, 2, 16, 16), (300000, 2, 16, 16),
+                                     (20000, 32, 1024, 64)])
 def test_layout_extreme_shapes(T, k, E, R):
     rng = np.random.default_rng(T + k + E)
     idx = np.argsort(rng.random((T, E)), axis=1)[:, :k] if E <= 64 else \
@@ -95,13 +98,15 @@ def test_layout_bad_ids_reported_and_dropped(T):
 
 
 def test_layout_workspace_reused_across_calls():
-    # the ticket in the workspace resets itself: one zeroed buffer serves
-    # many calls in stream order
-    cfg = workloads.CONFIGS["skewed"]
-    ws = torch.zeros(ep.ep_layout_workspace_bytes(cfg.T, cfg.k, cfg.E, cfg.R),
+    # tiled path: the ticket in the workspace resets itself, so one zeroed
+    # buffer serves many calls in stream order
+    cfg = workloads.CONFIGS["large"]
+    T = 70000
+    ws = torch.zeros(ep.ep_layout_workspace_bytes(T, cfg.k, cfg.E, cfg.R),
                      dtype=torch.uint8, device="cuda")
+    assert ws.numel() > 0
     for seed in range(3):
-        b = workloads.make_batch(cfg, seed, H=8)
+        b = workloads.make_batch(cfg, seed, T=T, H=8)
         L = ep.ep_get_layout(b.idx.cuda(), cfg.E, cfg.R, ws=ws)
         ref = oracle.layout(b.idx, cfg.E, cfg.R)
         np.testing.assert_array_equal(L.slot_pos.cpu().numpy(), ref["slot_pos"])
@@ -224,7 +229,9 @@ def _combine_check(cfg, b, sample=None, num_sms=0):
     assert_layout_equal(g, ref)
     y = workloads.expert_outputs(b.x, torch.from_numpy(ref["recv_src"]),
                                  torch.from_numpy(ref["off_e"]), cfg.expert)
-    out = ep.ep_combine(y.cuda(), L.slot_pos, b.w.cuda(), num_sms=num_sms)
+    d_err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = ep.ep_combine(y.cuda(), L.slot_pos, b.w.cuda(), num_sms=num_sms, d_err=d_err)
+    assert ep.ep_read_error(d_err) == 0
     got = tensor_bits16(out)
     if sample is None:
         want = oracle.combine(y, ref["slot_pos"], b.w)

@@ -32,13 +32,15 @@ def test_noalloc_matches_workspace_entry_point_two_calls_in_a_row():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     dev = torch.device("cuda")
-    # two different tiled-path batches back to back: the second call finds
-    # the first one's counters in the shared array
-    for name, seed in (("prefill", 0), ("skewed", 1)):
-        cfg = workloads.CONFIGS[name]
-        assert 0 < ep.ep_layout_workspace_bytes(cfg.T, cfg.k, cfg.E, cfg.R) \
+    # two different batches big enough for the tiled (scratch-using) layout,
+    # back to back: the second call finds the first one's counters in the
+    # shared array
+    cfg = workloads.CONFIGS["large"]
+    for T, seed in ((70000, 0), (66000, 1)):
+        assert 0 < ep.ep_layout_workspace_bytes(T, cfg.k, cfg.E, cfg.R) \
             <= ep.EP_NOALLOC_SCRATCH_BYTES
-        idx = workloads.make_batch(cfg, seed, H=8).idx.to(dev)
+        name = f"T={T}"
+        idx = workloads.make_batch(cfg, seed, T=T, H=8).idx.to(dev)
         want = ep.ep_get_layout(idx, cfg.E, cfg.R)
         got = ep.ep_get_layout_noalloc(idx, cfg.E, cfg.R)
         torch.cuda.synchronize()
