@@ -519,6 +519,51 @@ def bench_reference(args, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+def profile_kernel(args, device):
+    """Runs one kernel of the path by itself, --steps times after --warmup
+    warm-ups, with the L2 flush before each launch: the small, repeatable
+    command that Nsight Compute captures are taken on.  Prints the mean
+    CUDA-event time of the kernel (not a benchmark line)."""
+    import combine_ep_get_09_b200 as ep
+    cfg = workloads.CONFIGS[args.workload]
+    st = Step(ep, cfg, workloads.make_batch(cfg, seed=0), device)
+    stream = torch.cuda.Stream(device)
+    flush = L2Flush(device)
+    c = cfg
+    calls = {
+        "layout": lambda: ep.ep_get_layout(st.idx, c.E, c.R, out=st.layout, ws=st.ws,
+                                           d_err=st.d_err, stream=stream),
+        "dispatch_bf16": lambda: ep.ep_dispatch(st.x, st.layout.slot_pos, recv=st.recv,
+                                                d_err=st.d_err, stream=stream),
+        "dispatch_fp8": lambda: ep.ep_dispatch(st.x, st.layout.slot_pos, fp8=True,
+                                               recv=st.recv_q, recv_scale=st.recv_s,
+                                               d_err=st.d_err, stream=stream),
+        "combine": lambda: ep.ep_combine(st.recv, st.layout.slot_pos, st.w, out=st.out,
+                                         d_err=st.d_err, stream=stream),
+    }
+    call = calls[args.profile]
+    with torch.cuda.stream(stream):
+        st.run(stream)
+        for _ in range(args.warmup):
+            flush()
+            call()
+        ts = []
+        for _ in range(args.steps):
+            flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            ts.append((a, b))
+    stream.synchronize()
+    if ep.ep_read_error(st.d_err, stream) != 0:
+        raise RuntimeError("the device reported an error")
+    us = statistics.mean(a.elapsed_time(b) for a, b in ts) * 1e3
+    print(json.dumps({"profile": args.profile, "workload": args.workload,
+                      "launches_timed": args.steps, "us_mean": round(us, 2)}))
+
+
 def main():
     p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     p.add_argument("--gpus", type=int, default=1)
@@ -530,6 +575,10 @@ def main():
     p.add_argument("--skip-cpu", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--reference-tokens", type=int, default=256)
+    p.add_argument("--profile", choices=("layout", "dispatch_bf16", "dispatch_fp8", "combine"),
+                   help="run only this kernel (for profiler captures)")
+    p.add_argument("--workload", choices=tuple(workloads.CONFIGS), default="prefill",
+                   help="workload of --profile")
     args = p.parse_args()
     if args.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -545,6 +594,9 @@ def main():
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    if args.profile:
+        profile_kernel(args, device)
+        return
     if world > 1:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

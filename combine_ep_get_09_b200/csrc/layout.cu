@@ -5,20 +5,24 @@
 // Two paths, both deterministic (no ordering ever depends on atomics) and
 // neither with a CTA that waits on another through memory:
 //  * cluster (T*k <= kClusterMaxSlots): one launch of a thread-block
-//    cluster of up to 16 CTAs (1 CTA for small batches such as a 128-token
-//    decode step).  Each CTA counts its contiguous token range, the CTAs
-//    exchange their per-expert counts through distributed shared memory
-//    between two hardware cluster barriers, and every CTA then places its
-//    own slots.  No global workspace.
+//    cluster of up to 16 CTAs (a single plain CTA for small batches such as
+//    a 128-token decode step).  Each CTA ranks its contiguous token range,
+//    the CTAs exchange their per-expert counts through distributed shared
+//    memory between two hardware cluster barriers, and every CTA then
+//    places its own slots.  No global workspace.
 //  * tiled (larger batches): a counting kernel writes one histogram row per
 //    tile of tokens to the caller's workspace, and the last tile to finish
 //    (ticket taken with atomicInc, which wraps it back to 0) turns the rows
 //    into absolute per-tile bases and the global offsets; a placing kernel
-//    then gives every slot its row.
-// Inside a CTA each warp owns a contiguous run of slots.  Stable ranks
-// within 32 slots come from __match_any_sync + popc of the lower lanes; the
-// per-warp running bases come from per-warp histograms scanned across warps,
-// so slot order = token-major order exactly.
+//    then ranks and places every slot.
+//
+// Inside a CTA each warp owns a contiguous run of slots.  The lanes of a
+// 32-slot chunk that hold the same expert find each other with one ballot
+// per bit of the expert id (a slot's rank among them = popc of the lower
+// such lanes); each warp keeps running per-expert counts in its own row of
+// a shared histogram (row stride padded to avoid bank conflicts), and one
+// thread per expert scans the rows across warps.  Slot order is therefore
+// token-major order exactly.
 #include <cooperative_groups.h>
 
 #include <map>
@@ -35,7 +39,9 @@ constexpr int kClusterThreads = 1024;
 constexpr int kClusterWarps = kClusterThreads / kWarp;
 constexpr int kMaxClusterCtas = 16;
 constexpr long kClusterMaxSlots = 1L << 19;
-constexpr long kSlotsPerClusterCta = 4096;  // below this, fewer CTAs
+constexpr long kSlotsPerClusterCta = 2048;  // below this, fewer CTAs
+constexpr long kSmallSlots = 2048;          // one CTA of kSmallThreads
+constexpr int kSmallThreads = 256;
 
 constexpr int kTileThreads = 512;
 constexpr int kTileWarps = kTileThreads / kWarp;
@@ -45,7 +51,9 @@ constexpr int kTicketBytes = 16;
 
 struct Params {
   const void *idx;
-  int T, k, E, R, G;
+  int T, k, E, R;
+  int id_bits;                 // bits of an expert id: 2^id_bits >= E
+  unsigned long long g_magic;  // ceil(2^32 / G): e / G == (e * g_magic) >> 32 for e < 1024
   int32_t *cnt_e, *cnt_r, *off_e, *off_r, *slot_pos, *recv_src;
   uint8_t *in_rank;
   int32_t *d_err;
@@ -60,6 +68,10 @@ __device__ __forceinline__ int check_id(long long e, int E, int32_t *d_err) {
   if (e >= 0 && e < E) return static_cast<int>(e);
   if (e != -1 && d_err != nullptr) atomicExch(reinterpret_cast<int *>(d_err), EP_ERR_INDEX);
   return -1;
+}
+
+__device__ __forceinline__ int rank_of(int e, const Params &p) {
+  return static_cast<int>((static_cast<unsigned long long>(e) * p.g_magic) >> 32);
 }
 
 // Ids are read kIdBatch at a time per lane, all loads issued before any is
@@ -77,44 +89,6 @@ __device__ __forceinline__ void load_id_batch(const IdT *idx, long c0, long end,
   }
 }
 
-// In-place exclusive scan of a[0..n) in shared memory by the whole block;
-// returns the total.  warp_tmp: 32 ints of shared memory.
-__device__ int block_exclusive_scan(int *a, int n, int *warp_tmp) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
-  const int per = (n + nt - 1) / nt;
-  const int beg = min(n, tid * per), end = min(n, beg + per);
-  int local = 0;
-  for (int i = beg; i < end; ++i) local += a[i];
-  int v = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += u;
-  }
-  if (lane == 31) warp_tmp[wid] = v;
-  __syncthreads();
-  if (wid == 0) {
-    int t = lane < nw ? warp_tmp[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += u;
-    }
-    if (lane < nw) warp_tmp[lane] = t;
-  }
-  __syncthreads();
-  int run = v - local + (wid > 0 ? warp_tmp[wid - 1] : 0);
-  const int total = warp_tmp[nw - 1];
-  for (int i = beg; i < end; ++i) {
-    const int c = a[i];
-    a[i] = run;
-    run += c;
-  }
-  __syncthreads();
-  return total;
-}
-
 // Contiguous, 32-aligned slice [b, *end) of [0, n) for warp w of nw.
 __device__ __forceinline__ long warp_slice(long n, int w, int nw, long *end) {
   const long s = ((n + nw - 1) / nw + 31) / 32 * 32;
@@ -123,85 +97,211 @@ __device__ __forceinline__ long warp_slice(long n, int w, int nw, long *end) {
   return b;
 }
 
-// Per-warp counts of the kept ids in slots [beg, end) (warp-uniform range).
-template <typename IdT>
-__device__ void count_segment(const IdT *idx, long beg, long end, int E, int32_t *d_err,
-                              int *hist_w) {
-  for (long c0 = beg; c0 < end; c0 += 32 * kIdBatch) {
-    long long v[kIdBatch];
-    load_id_batch(idx, c0, end, v);
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int b = 0; b < kIdBatch; ++b) {
-      const int e = check_id(v[b], E, d_err);
-      if (e >= 0) atomicAdd(&hist_w[e], 1);
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
+// Exclusive scan of a[0..n) in shared memory by one warp (each lane owns a
+// contiguous run); returns the total to every lane.
+__device__ int warp_exclusive_scan_smem(int *a, int n) {
+  const int lane = threadIdx.x & 31;
+  const int per = (n + 31) / 32;
+  const int beg = min(n, lane * per), end = min(n, beg + per);
+  int local = 0;
+  for (int i = beg; i < end; ++i) local += a[i];
+  const int incl = warp_inclusive_scan(local);
+  int run = incl - local;
+  for (int i = beg; i < end; ++i) {
+    const int c = a[i];
+    a[i] = run;
+    run += c;
+  }
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// Lanes of the warp whose key equals this lane's, among the lanes in
+// `valid`: the intersection over the key's bits of the lanes that agree on
+// each bit (one ballot per bit).
+__device__ __forceinline__ unsigned match_key(int key, int bits, unsigned valid) {
+  unsigned peers = valid;
+  for (int b = 0; b < bits; ++b) {
+    const unsigned ones = __ballot_sync(0xffffffffu, (key >> b) & 1);
+    peers &= ((key >> b) & 1) ? ones : ~ones;
+  }
+  return peers;
+}
+
+// Per-warp histograms: row w holds warp w's counts, columns [0, E) experts
+// and [E, E + R) ranks; the row stride E + R + 1 keeps the threads of one
+// column scan on distinct banks.
+__device__ __forceinline__ int hist_ld(const Params &p) { return p.E + p.R + 1; }
+
+// For each column c of the nw rows, one thread: hist[w][c] becomes the
+// count of the earlier warps (experts only) and total[c] the CTA's count.
+__device__ void scan_hist_columns(int *hist, int ld, int E, int C, int nw, int *total) {
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    int run = 0;
+    for (int v = 0; v < nw; ++v) {
+      const int x = hist[v * ld + c];
+      if (c < E) hist[v * ld + c] = run;
+      run += x;
     }
+    total[c] = run;
   }
 }
 
-// Gives each slot in [beg, end) its row; base[e] holds the next free row of
-// expert e for this warp and is advanced as slots are placed.
-template <typename IdT>
-__device__ void place_segment(const IdT *idx, long beg, long end, int k, int E, int *base,
-                              int32_t *slot_pos, int32_t *recv_src) {
-  const int lane = threadIdx.x & 31;
+// hist[w][e] += base[e] for every warp w (base: the expert's first row for
+// this CTA), one thread per expert.
+__device__ void add_column_bases(int *hist, int ld, int E, int nw, const int *base) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int b = base[e];
+    for (int v = 0; v < nw; ++v) hist[v * ld + e] += b;
+  }
+}
+
+// A warp's stable ranking of its slot segment [beg, end).
+//
+// Pass 1 (rank_segment) walks the segment 32 slots at a time: a slot's rank
+// among the warp's slots of its expert is the warp's running count of that
+// expert (hist_w[e], zeroed by the caller) plus the number of lower lanes
+// holding the same expert.  The first kRegChunks chunks keep expert and
+// rank in registers (packed as rank << 10 | e, -1 for no kept slot; E <=
+// 1024); later chunks park the rank in the slot_pos output.  At the end
+// hist_w[e] is the warp's count of e.
+//
+// Pass 2 (place_segment) turns ranks into rows, base_w[e] being the
+// warp's first row of expert e, and writes slot_pos and recv_src.
+constexpr int kRegChunks = kIdBatch;
+
+struct SegRanks {
+  int packed[kRegChunks];
+};
+
+__device__ __forceinline__ int rank_one(int e, int bits, int *hist_w) {
   const unsigned lt = lanemask_lt();
-  for (long c0 = beg; c0 < end; c0 += 32 * kIdBatch) {
+  const unsigned valid = __ballot_sync(0xffffffffu, e >= 0);
+  const unsigned peers = match_key(e, bits, valid);
+  const int r = e >= 0 ? hist_w[e] + __popc(peers & lt) : -1;
+  __syncwarp();
+  if (e >= 0 && (peers & lt) == 0) hist_w[e] += __popc(peers);
+  __syncwarp();
+  return r;
+}
+
+template <typename IdT>
+__device__ void rank_segment(const IdT *idx, long beg, long end, int E, int bits,
+                             int32_t *d_err, int *hist_w, int32_t *slot_pos, SegRanks &sr) {
+  const int lane = threadIdx.x & 31;
+  {
+    long long v[kIdBatch];
+    load_id_batch(idx, beg, end, v);
+#pragma unroll
+    for (int b = 0; b < kRegChunks; ++b) {
+      sr.packed[b] = -1;
+      if (beg + 32 * b < end) {  // uniform across the warp
+        const int e = check_id(v[b], E, d_err);
+        const int r = rank_one(e, bits, hist_w);
+        sr.packed[b] = e >= 0 ? (r << 10) | e : -1;
+      }
+    }
+  }
+  for (long c0 = beg + 32 * kRegChunks; c0 < end; c0 += 32 * kIdBatch) {
     long long v[kIdBatch];
     load_id_batch(idx, c0, end, v);
 #pragma unroll
     for (int b = 0; b < kIdBatch; ++b) {
       if (c0 + 32 * b >= end) break;  // uniform across the warp
       const long i = c0 + 32 * b + lane;
-      const int e = check_id(v[b], E, nullptr);
-      // lanes without a kept slot get keys no other lane can share
-      const int key = e >= 0 ? e : -2 - lane;
-      const unsigned peers = __match_any_sync(0xffffffffu, key);
-      int pos = -1;
-      if (e >= 0) {
-        pos = base[e] + __popc(peers & lt);
-        recv_src[pos] = static_cast<int32_t>(i / k);
-      }
-      if (i < end) slot_pos[i] = pos;
-      __syncwarp();
-      if (e >= 0 && (peers & lt) == 0) base[e] += __popc(peers);
-      __syncwarp();
+      const int r = rank_one(check_id(v[b], E, d_err), bits, hist_w);
+      if (i < end) slot_pos[i] = r;
     }
   }
 }
 
-// Token-in-rank mask rows for tokens [t_beg, t_end) and their per-rank
-// counts (atomics into rank_cnt[R]: counts only, no order involved).
 template <typename IdT>
-__device__ void rank_mask(const Params &p, int t_beg, int t_end, int *rank_cnt) {
-  const IdT *idx = static_cast<const IdT *>(p.idx);
-  for (int t = t_beg + threadIdx.x; t < t_end; t += blockDim.x) {
-    const long base = static_cast<long>(t) * p.k;
-    unsigned long long m = 0;
-    for (int j0 = 0; j0 < p.k; j0 += kIdBatch) {
-      long long v[kIdBatch];
+__device__ void place_segment(const IdT *idx, long beg, long end, int k, int E,
+                              const int *base_w, const SegRanks &sr, int32_t *slot_pos,
+                              int32_t *recv_src) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-      for (int b = 0; b < kIdBatch; ++b)
-        v[b] = j0 + b < p.k ? static_cast<long long>(idx[base + j0 + b]) : -1;
+  for (int b = 0; b < kRegChunks; ++b) {
+    const long i = beg + 32 * b + lane;
+    if (i < end) {
+      const int q = sr.packed[b];
+      const int pos = q >= 0 ? base_w[q & 1023] + (q >> 10) : -1;
+      slot_pos[i] = pos;
+      if (pos >= 0) recv_src[pos] = static_cast<int32_t>(i / k);
+    }
+  }
+  for (long c0 = beg + 32 * kRegChunks; c0 < end; c0 += 32 * kIdBatch) {
+    long long v[kIdBatch];
+    load_id_batch(idx, c0, end, v);
 #pragma unroll
-      for (int b = 0; b < kIdBatch; ++b) {
-        const int e = check_id(v[b], p.E, nullptr);
-        if (e >= 0) m |= 1ull << (e / p.G);
+    for (int b = 0; b < kIdBatch; ++b) {
+      const long i = c0 + 32 * b + lane;
+      if (i < end) {
+        const int e = check_id(v[b], E, nullptr);
+        const int pos = e >= 0 ? base_w[e] + slot_pos[i] : -1;
+        slot_pos[i] = pos;
+        if (pos >= 0) recv_src[pos] = static_cast<int32_t>(i / k);
       }
     }
-    uint8_t *row = p.in_rank + static_cast<long>(t) * p.R;
-    for (int r = 0; r < p.R; ++r) row[r] = static_cast<uint8_t>((m >> r) & 1u);
-    while (m) {
-      const int r = __ffsll(static_cast<long long>(m)) - 1;
-      atomicAdd(&rank_cnt[r], 1);
-      m &= m - 1;
+  }
+}
+
+// Token-in-rank mask rows for tokens [t_beg, t_end).  Per-rank token counts
+// go into this warp's histogram row, columns E..E+R-1 (one ballot per rank,
+// written by lane 0: the row is the warp's own).  Every thread of the
+// block runs the same number of rounds.
+template <typename IdT>
+__device__ void rank_mask(const Params &p, int t_beg, int t_end, int *hist_w) {
+  const IdT *idx = static_cast<const IdT *>(p.idx);
+  const int lane = threadIdx.x & 31;
+  for (int t0 = t_beg; t0 < t_end; t0 += blockDim.x) {
+    const int t = t0 + threadIdx.x;
+    unsigned long long m = 0;
+    if (t < t_end) {
+      const long base = static_cast<long>(t) * p.k;
+      for (int j0 = 0; j0 < p.k; j0 += kIdBatch) {
+        long long v[kIdBatch];
+#pragma unroll
+        for (int b = 0; b < kIdBatch; ++b)
+          v[b] = j0 + b < p.k ? static_cast<long long>(idx[base + j0 + b]) : -1;
+#pragma unroll
+        for (int b = 0; b < kIdBatch; ++b) {
+          const int e = check_id(v[b], p.E, nullptr);
+          if (e >= 0) m |= 1ull << rank_of(e, p);
+        }
+      }
+      uint8_t *row = p.in_rank + static_cast<long>(t) * p.R;
+      if ((p.R & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 3) == 0) {
+        // 4 mask bytes per 32-bit store
+        for (int r = 0; r < p.R; r += 4) {
+          const unsigned b = static_cast<unsigned>(m >> r);
+          reinterpret_cast<uint32_t *>(row)[r >> 2] =
+              (b & 1u) | ((b >> 1) & 1u) << 8 | ((b >> 2) & 1u) << 16 | ((b >> 3) & 1u) << 24;
+        }
+      } else {
+        for (int r = 0; r < p.R; ++r) row[r] = static_cast<uint8_t>((m >> r) & 1u);
+      }
+    }
+    for (int r = 0; r < p.R; ++r) {
+      const unsigned bal = __ballot_sync(0xffffffffu, (m >> r) & 1u);
+      if (lane == 0) hist_w[p.E + r] += __popc(bal);
     }
   }
 }
 
 // ------------------------------------------------------------- cluster path
 
-int cluster_smem_bytes(int E, int R) {
-  return (kClusterWarps * E + 3 * (E + R) + 32) * static_cast<int>(sizeof(int));
+int cluster_smem_bytes(int E, int R, int warps) {
+  return (warps * (E + R + 1) + 4 * (E + R)) * static_cast<int>(sizeof(int));
 }
 
 template <typename IdT>
@@ -210,14 +310,15 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
   const int n_ctas = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   extern __shared__ int smem[];
-  const int E = p.E, R = p.R, C = E + R;
-  int *hist = smem;                       // [warps][E]
-  int *mine = hist + kClusterWarps * E;   // [C] this CTA's counts, read by all CTAs
-  int *before = mine + C;                 // [C] counts of the lower-ranked CTAs
-  int *tot = before + C;                  // [C] totals, then exclusive offsets
-  int *warp_tmp = tot + C;                // [32]
+  const int E = p.E, R = p.R, C = E + R, ld = hist_ld(p);
+  const int tid = threadIdx.x, nt = blockDim.x, w = tid >> 5, nw = nt >> 5;
+  int *hist = smem;            // [warps][E + R + 1]
+  int *mine = hist + nw * ld;  // [C] this CTA's counts, read by all CTAs
+  int *before = mine + C;      // [C] counts of the lower-ranked CTAs
+  int *tot = before + C;       // [C] totals, then exclusive offsets
+  int *base = tot + C;         // [C] first row of each expert for this CTA
+  __shared__ int s_kept;       // rows in use (all CTAs)
   const IdT *idx = static_cast<const IdT *>(p.idx);
-  const int tid = threadIdx.x, nt = blockDim.x, w = tid >> 5;
 
   const int per_cta = (p.T + n_ctas - 1) / n_ctas;
   const int t_beg = min(p.T, rank * per_cta);
@@ -225,62 +326,75 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
   const long s_beg = static_cast<long>(t_beg) * p.k;
   const long n = static_cast<long>(t_end - t_beg) * p.k;
 
-  for (int i = tid; i < kClusterWarps * E + C; i += nt) smem[i] = 0;
+  for (int i = tid; i < nw * ld; i += nt) smem[i] = 0;
   __syncthreads();
   long seg_end;
-  const long seg_beg = warp_slice(n, w, kClusterWarps, &seg_end);
-  count_segment(idx, s_beg + seg_beg, s_beg + seg_end, E, p.d_err, hist + w * E);
-  rank_mask<IdT>(p, t_beg, t_end, mine + E);
+  const long seg_beg = warp_slice(n, w, nw, &seg_end);
+  SegRanks sr;
+  rank_segment(idx, s_beg + seg_beg, s_beg + seg_end, E, p.id_bits, p.d_err, hist + w * ld,
+               p.slot_pos, sr);
+  rank_mask<IdT>(p, t_beg, t_end, hist + w * ld);
   __syncthreads();
-  // hist[w][e] -> count of the earlier warps; mine[e] -> this CTA's total
-  for (int e = tid; e < E; e += nt) {
-    int run = 0;
-    for (int v = 0; v < kClusterWarps; ++v) {
-      const int c = hist[v * E + e];
-      hist[v * E + e] = run;
-      run += c;
+  scan_hist_columns(hist, ld, E, C, nw, mine);  // mine[c] = this CTA's count
+  if (n_ctas > 1) {
+    cluster.sync();  // every CTA's `mine` is complete and visible
+    for (int c = tid; c < C; c += nt) {
+      int b = 0, a = 0;
+      for (int r0 = 0; r0 < n_ctas; r0 += 8) {
+        int v[8];  // 8 remote loads in flight
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          v[u] = r0 + u < n_ctas ? cluster.map_shared_rank(mine, r0 + u)[c] : 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          b += r0 + u < rank ? v[u] : 0;
+          a += v[u];
+        }
+      }
+      before[c] = b;
+      tot[c] = a;
     }
-    mine[e] = run;
-  }
-  cluster.sync();  // every CTA's `mine` is complete and visible
-  for (int c = tid; c < C; c += nt) {
-    int b = 0, a = 0;
-    for (int r = 0; r < n_ctas; ++r) {
-      const int v = cluster.map_shared_rank(mine, r)[c];
-      b += r < rank ? v : 0;
-      a += v;
+    cluster.sync();  // no CTA reads another's shared memory after this
+  } else {
+    __syncthreads();
+    for (int c = tid; c < C; c += nt) {
+      before[c] = 0;
+      tot[c] = mine[c];
     }
-    before[c] = b;
-    tot[c] = a;
+    __syncthreads();
   }
-  cluster.sync();  // no CTA reads another's shared memory after this
   if (rank == 0)
     for (int c = tid; c < C; c += nt) {
       if (c < E) p.cnt_e[c] = tot[c];
       else p.cnt_r[c - E] = tot[c];
     }
+  // warp 0 scans the expert totals, warp 1 the rank totals
+  if (w == 0) {
+    const int n_kept = warp_exclusive_scan_smem(tot, E);
+    if (tid == 0) {
+      s_kept = n_kept;
+      if (rank == 0) p.off_e[E] = n_kept;
+    }
+  } else if (w == 1) {
+    const int n_tok = warp_exclusive_scan_smem(tot + E, R);
+    if (rank == 0 && (tid & 31) == 0) p.off_r[R] = n_tok;
+  }
   __syncthreads();
-  const int n_kept = block_exclusive_scan(tot, E, warp_tmp);
-  const int n_tok = block_exclusive_scan(tot + E, R, warp_tmp);
-  if (rank == 0) {
-    for (int c = tid; c < C; c += nt) {
+  for (int c = tid; c < C; c += nt) {
+    if (rank == 0) {
       if (c < E) p.off_e[c] = tot[c];
       else p.off_r[c - E] = tot[c];
     }
-    if (tid == 0) {
-      p.off_e[E] = n_kept;
-      p.off_r[R] = n_tok;
-    }
-  }
-  for (int e = tid; e < E; e += nt) {
-    const int b = tot[e] + before[e];
-    for (int v = 0; v < kClusterWarps; ++v) hist[v * E + e] += b;
+    if (c < E) base[c] = tot[c] + before[c];
   }
   __syncthreads();
-  place_segment(idx, s_beg + seg_beg, s_beg + seg_end, p.k, E, hist + w * E, p.slot_pos,
+  add_column_bases(hist, ld, E, nw, base);
+  __syncthreads();
+  place_segment(idx, s_beg + seg_beg, s_beg + seg_end, p.k, E, hist + w * ld, sr, p.slot_pos,
                 p.recv_src);
+  // rows nobody fills (past the kept ones)
   const long N = static_cast<long>(p.T) * p.k;
-  for (long r = n_kept + static_cast<long>(rank) * nt + tid; r < N;
+  for (long r = s_kept + static_cast<long>(rank) * nt + tid; r < N;
        r += static_cast<long>(n_ctas) * nt)
     p.recv_src[r] = -1;
 }
@@ -290,21 +404,22 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
 template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
   extern __shared__ int smem[];
-  const int E = p.E, R = p.R, C = E + R;
-  const int tid = threadIdx.x, nt = blockDim.x;
-  int *col = smem;                    // [C]   this tile's counts, later totals
+  const int E = p.E, R = p.R, C = E + R, ld = hist_ld(p);
+  const int tid = threadIdx.x, nt = blockDim.x, w = tid >> 5, nw = nt >> 5;
+  int *hist = smem;                   // [warps][E + R + 1] per-warp counts
+  int *col = hist + nw * ld;          // [C] this tile's counts, later totals
   int *part = col + C;                // [max(nt, C)] partial column sums
-  int *warp_tmp = part + max(nt, C);  // [32]
-  int *flag = warp_tmp + 32;          // [1]
+  int *flag = part + max(nt, C);      // [1]
   const IdT *idx = static_cast<const IdT *>(p.idx);
   const int tile = blockIdx.x;
   const int t_beg = tile * p.tile_T;
   const int t_end = min(p.T, t_beg + p.tile_T);
 
-  for (int i = tid; i < C; i += nt) col[i] = 0;
+  for (int i = tid; i < nw * ld; i += nt) hist[i] = 0;
   __syncthreads();
   const long s_end = static_cast<long>(t_end) * p.k;
-  for (long c0 = static_cast<long>(t_beg) * p.k; c0 < s_end; c0 += static_cast<long>(nt) * kIdBatch) {
+  for (long c0 = static_cast<long>(t_beg) * p.k; c0 < s_end;
+       c0 += static_cast<long>(nt) * kIdBatch) {
     long long v[kIdBatch];
 #pragma unroll
     for (int b = 0; b < kIdBatch; ++b) {
@@ -314,10 +429,12 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
 #pragma unroll
     for (int b = 0; b < kIdBatch; ++b) {
       const int e = check_id(v[b], E, p.d_err);
-      if (e >= 0) atomicAdd(&col[e], 1);
+      if (e >= 0) atomicAdd(&hist[w * ld + e], 1);
     }
   }
-  rank_mask<IdT>(p, t_beg, t_end, col + E);
+  rank_mask<IdT>(p, t_beg, t_end, hist + w * ld);
+  __syncthreads();
+  scan_hist_columns(hist, ld, E, C, nw, col);
   __syncthreads();
   for (int c = tid; c < C; c += nt) p.cols[static_cast<long>(tile) * C + c] = col[c];
 
@@ -359,15 +476,17 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
     else p.cnt_r[c - E] = s;
   }
   __syncthreads();
-  const int n_kept = block_exclusive_scan(col, E, warp_tmp);
-  const int n_tok = block_exclusive_scan(col + E, R, warp_tmp);
+  if (w == 0) {
+    const int n_kept = warp_exclusive_scan_smem(col, E);
+    if (tid == 0) p.off_e[E] = n_kept;
+  } else if (w == 1) {
+    const int n_tok = warp_exclusive_scan_smem(col + E, R);
+    if ((tid & 31) == 0) p.off_r[R] = n_tok;
+  }
+  __syncthreads();
   for (int c = tid; c < C; c += nt) {
     if (c < E) p.off_e[c] = col[c];
     else p.off_r[c - E] = col[c];
-  }
-  if (tid == 0) {
-    p.off_e[E] = n_kept;
-    p.off_r[R] = n_tok;
   }
   // absolute row base of every (tile, expert), in place
   for (int q = tid; q < C * P; q += nt) {
@@ -394,32 +513,33 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
 template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads) layout_place_kernel(Params p) {
   extern __shared__ int smem[];
-  const int E = p.E, C = p.E + p.R;
-  int *hist = smem;  // [warps][E]
-  const IdT *idx = static_cast<const IdT *>(p.idx);
+  const int E = p.E, C = p.E + p.R, ld = hist_ld(p);
   const int tid = threadIdx.x, w = tid >> 5;
+  int *hist = smem;                    // [warps][E + R + 1]
+  int *base = hist + kTileWarps * ld;  // [E] the tile's first row of each expert
+  int *scratch = base + E;             // [C] tile totals (unused)
+  const IdT *idx = static_cast<const IdT *>(p.idx);
   const int tile = blockIdx.x;
   const int t_beg = tile * p.tile_T;
   const int t_end = min(p.T, t_beg + p.tile_T);
   const long s_beg = static_cast<long>(t_beg) * p.k;
   const long n = static_cast<long>(t_end - t_beg) * p.k;
 
-  for (int i = tid; i < kTileWarps * E; i += blockDim.x) hist[i] = 0;
+  for (int i = tid; i < kTileWarps * ld; i += blockDim.x) hist[i] = 0;
+  for (int e = tid; e < E; e += blockDim.x)
+    base[e] = __ldcg(&p.cols[static_cast<long>(tile) * C + e]);
   __syncthreads();
   long seg_end;
   const long seg_beg = warp_slice(n, w, kTileWarps, &seg_end);
-  count_segment(idx, s_beg + seg_beg, s_beg + seg_end, E, nullptr, hist + w * E);
+  SegRanks sr;
+  rank_segment(idx, s_beg + seg_beg, s_beg + seg_end, E, p.id_bits, nullptr, hist + w * ld,
+               p.slot_pos, sr);
   __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) {
-    int run = __ldcg(&p.cols[static_cast<long>(tile) * C + e]);
-    for (int v = 0; v < kTileWarps; ++v) {
-      const int c = hist[v * E + e];
-      hist[v * E + e] = run;
-      run += c;
-    }
-  }
+  scan_hist_columns(hist, ld, E, E, kTileWarps, scratch);
   __syncthreads();
-  place_segment(idx, s_beg + seg_beg, s_beg + seg_end, p.k, E, hist + w * E, p.slot_pos,
+  add_column_bases(hist, ld, E, kTileWarps, base);
+  __syncthreads();
+  place_segment(idx, s_beg + seg_beg, s_beg + seg_end, p.k, E, hist + w * ld, sr, p.slot_pos,
                 p.recv_src);
 
   // rows nobody fills
@@ -477,17 +597,24 @@ int max_cluster_ctas(int smem) {
 template <typename IdT>
 cudaError_t launch_cluster(Params p, cudaStream_t s, int *launches) {
   auto kern = layout_cluster_kernel<IdT>;
-  const int smem = cluster_smem_bytes(p.E, p.R);
-  cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
-  if (err != cudaSuccess) return err;
   const long N = static_cast<long>(p.T) * p.k;
+  const int threads = N <= kSmallSlots ? kSmallThreads : kClusterThreads;
+  const int smem = cluster_smem_bytes(p.E, p.R, threads / kWarp);
+  cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern),
+                                       cluster_smem_bytes(p.E, p.R, kClusterWarps));
+  if (err != cudaSuccess) return err;
   long want = (N + kSlotsPerClusterCta - 1) / kSlotsPerClusterCta;
   if (want < 1) want = 1;
   const int cap = want > 8 ? max_cluster_ctas<IdT>(smem) : 8;
   const int n_ctas = static_cast<int>(want < cap ? want : cap);
+  ++*launches;
+  if (n_ctas == 1) {  // a plain launch: the kernel sees a cluster of one
+    kern<<<1, threads, smem, s>>>(p);
+    return cudaGetLastError();
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_ctas);
-  cfg.blockDim = dim3(kClusterThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr;
@@ -497,19 +624,19 @@ cudaError_t launch_cluster(Params p, cudaStream_t s, int *launches) {
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kern, p);
-  ++*launches;
-  return err;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 template <typename IdT>
 cudaError_t launch_tiled(Params p, cudaStream_t s, int *launches) {
-  const int C = p.E + p.R;
-  const int count_smem =
-      (C + (kTileThreads > C ? kTileThreads : C) + 32 + 1) * static_cast<int>(sizeof(int));
-  const int place_smem = kTileWarps * p.E * static_cast<int>(sizeof(int));
+  const int C = p.E + p.R, ld = p.E + p.R + 1;
+  const int count_smem = (kTileWarps * ld + C + (kTileThreads > C ? kTileThreads : C) + 1) *
+                         static_cast<int>(sizeof(int));
+  const int place_smem = (kTileWarps * ld + p.E + C) * static_cast<int>(sizeof(int));
   cudaError_t err =
-      raise_dynamic_smem(reinterpret_cast<const void *>(layout_place_kernel<IdT>), place_smem);
+      raise_dynamic_smem(reinterpret_cast<const void *>(layout_count_kernel<IdT>), count_smem);
+  if (err != cudaSuccess) return err;
+  err = raise_dynamic_smem(reinterpret_cast<const void *>(layout_place_kernel<IdT>), place_smem);
   if (err != cudaSuccess) return err;
   layout_count_kernel<IdT><<<p.ntiles, kTileThreads, count_smem, s>>>(p);
   ++*launches;
@@ -536,7 +663,10 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s, int *launches) {
   p.k = a.k;
   p.E = a.E;
   p.R = a.R;
-  p.G = a.E / a.R;
+  const int G = a.E / a.R;
+  p.g_magic = ((1ull << 32) + G - 1) / G;
+  p.id_bits = 0;
+  while ((1 << p.id_bits) < a.E) ++p.id_bits;
   p.cnt_e = a.cnt_e;
   p.cnt_r = a.cnt_r;
   p.off_e = a.off_e;
