@@ -194,6 +194,18 @@ def sum_over_ranks(v: float, world: int, device) -> float:
     return float(t.item())
 
 
+def rank_seed(rank: int) -> int:
+    """Seed of rank `rank`'s batch: every rank draws its own independent
+    batch of the workload (weak scaling: the work per GPU is fixed)."""
+    return rank
+
+
+def job_value(bytes_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job GB/s: the bytes all ranks moved over the slowest rank's
+    time."""
+    return world * bytes_per_rank_step * steps / (max_ms * 1e-3) / 1e9
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -251,7 +263,7 @@ def bench_ours(args, world, rank, device):
     import combine_ep_get_09_b200 as ep
     ep.lib()
     cfg = workloads.CONFIGS["prefill"]
-    batch = workloads.make_batch(cfg, seed=rank)
+    batch = workloads.make_batch(cfg, seed=rank_seed(rank))
     st = Step(ep, cfg, batch, device)
     stream = torch.cuda.Stream(device)
     flush = L2Flush(device)
@@ -301,7 +313,7 @@ def bench_ours(args, world, rank, device):
     dom_gbs = nbytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
     traffic = profiled_traffic(dom)
 
-    value = world * total_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    value = job_value(total_bytes, args.steps, world, total_ms)
     result = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -344,10 +356,30 @@ def bench_ours(args, world, rank, device):
     return result
 
 
+# Library sources each kernel is built from: a profile's DRAM traffic is
+# only reported while these files are byte-for-byte the ones profiled.
+KERNEL_SOURCES = {
+    "layout": ("layout.cu", "ep_internal.cuh"),
+    "dispatch_bf16": ("dispatch.cu", "ep_internal.cuh"),
+    "dispatch_fp8": ("dispatch.cu", "ep_internal.cuh"),
+    "combine": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),
+}
+
+
+def kernel_source_digest(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "combine_ep_get_09_b200", "csrc", name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def profiled_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary of `kernel`,
-    valid only while the library sources are the ones profiled."""
-    from combine_ep_get_09_b200 import build as lib_build
+    """DRAM bytes per launch (read + write) from the committed Nsight Compute
+    summary profiles/<kernel>_prefill.md, or None when there is none or the
+    kernel's sources changed since it was taken."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_prefill.md")
     try:
         with open(path) as f:
@@ -356,7 +388,7 @@ def profiled_traffic(kernel: str):
         return None
     m = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
     t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m or not t or m.group(1) != lib_build.source_digest():
+    if not m or not t or m.group(1) != kernel_source_digest(kernel):
         return None
     return float(t.group(1))
 
@@ -445,7 +477,7 @@ def bench_e2e(ep, cfg, batch, device, args, world, total_bytes):
     ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), world, device)
     h2d = h_idx.numel() * 8 + h_w.numel() * 4 + h_x.numel() * 2
     d2h = h_out.numel() * 2
-    return {"value": round(world * total_bytes * n / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+    return {"value": round(job_value(total_bytes, n, world, ms), 1), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / n, 4), "steps": n}
 
