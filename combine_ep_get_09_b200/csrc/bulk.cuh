@@ -80,6 +80,13 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, 
 }
 
 // Shared -> global bulk copy in the current bulk async-group.
+__device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src, unsigned bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+               "r"(smem_addr(smem_src)), "r"(bytes)
+               : "memory");
+}
+
+// The same with an L2 policy.
 __device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src, unsigned bytes,
                                            uint64_t policy) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(

@@ -66,12 +66,14 @@ __global__ void __launch_bounds__(kChunkVec)
   const long first = min(items, static_cast<long>(blockIdx.x) * per_cta);
   const long n_mine = min(items, first + per_cta) - first;
 
+  pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
     mbar_init_fence();
     timed_out = 0;
   }
   __syncthreads();
+  pdl_wait();
 
   // thread 0: gather item i's slot rows into stage i % kStages
   auto issue = [&](long i) {
@@ -141,6 +143,8 @@ __global__ void __launch_bounds__(kRegThreads, 2)
     combine_reg_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
                        const int32_t *__restrict__ slot_pos, const float *__restrict__ w,
                        uint4 *__restrict__ out, long n_rows) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int nchunks = (Hv + 31) / 32;
   const long items = static_cast<long>(T) * nchunks;
@@ -195,20 +199,19 @@ cudaError_t launch_combine(const void *y, int T, int H, int k, const int32_t *sl
     const long grid = persistent_grid(reinterpret_cast<const void *>(combine_bulk_kernel),
                                       kChunkVec, kBulkSmem, items * (kChunkVec / kWarp),
                                       num_sms);
-    combine_bulk_kernel<<<grid, kChunkVec, kBulkSmem, s>>>(
-        static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w, static_cast<uint4 *>(out), n_rows,
-        d_err);
     ++*launches;
-    return cudaGetLastError();
+    return launch_pdl(combine_bulk_kernel, dim3(grid), dim3(kChunkVec), kBulkSmem, s, 1,
+                      static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,
+                      static_cast<uint4 *>(out), n_rows, d_err);
   }
   const long items = static_cast<long>(T) * ((Hv + 31) / 32);
   if (items == 0) return cudaSuccess;
   const long grid = persistent_grid(reinterpret_cast<const void *>(combine_reg_kernel),
                                     kRegThreads, 0, items, num_sms);
-  combine_reg_kernel<<<grid, kRegThreads, 0, s>>>(static_cast<const uint4 *>(y), T, Hv, k,
-                                                  slot_pos, w, static_cast<uint4 *>(out), n_rows);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(combine_reg_kernel, dim3(grid), dim3(kRegThreads), 0, s, 1,
+                    static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,
+                    static_cast<uint4 *>(out), n_rows);
 }
 
 }  // namespace ep

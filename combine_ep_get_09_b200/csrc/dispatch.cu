@@ -9,6 +9,7 @@
 // are fetched by lanes 0..k-1 and broadcast with shuffles.
 #include <cuda_fp8.h>
 
+#include "bulk.cuh"
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -22,6 +23,8 @@ __global__ void __launch_bounds__(kThreads)
     dispatch_bf16_kernel(const uint4 *__restrict__ x, int T, int Hv, int k,
                          const int32_t *__restrict__ slot_pos,
                          uint4 *__restrict__ recv, long n_rows) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int per_chunk = 32 * V;
   const int nchunks = (Hv + per_chunk - 1) / per_chunk;
@@ -75,6 +78,107 @@ __device__ __forceinline__ uint2 quantize_bf16x8(uint4 v, float s) {
   return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
 }
 
+// amax -> scale -> e4m3 for the 8 bf16 values of one lane, the lane being
+// one of the 16 lanes (a half-warp) that hold a 128-channel block.
+__device__ __forceinline__ uint2 quantize_block_lane(uint4 v, float *scale) {
+  uint32_t m = absmax_bits_bf16x8(v);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float a = __uint_as_float(m << 16);
+  a = a < 1e-4f ? 1e-4f : a;  // keeps NaN
+  *scale = __fdiv_rn(a, 448.0f);
+  return quantize_bf16x8(v, *scale);
+}
+
+constexpr int kFp8BulkThreads = 256;
+constexpr int kFp8BulkStages = 2;  // input rows in flight per CTA
+
+// FP8 dispatch through shared memory, one whole token row per item (H a
+// multiple of 512, so both the e4m3 row and its H/128 scales are whole
+// 16-byte units): thread 0 bulk-loads the next token's bf16 row while the
+// CTA quantizes the current one into an output stage (half-warp per
+// 128-channel block), then thread 0 bulk-stores that stage to each of the
+// token's k receive rows (payload and scales).  Bulk stores of whole rows
+// write HBM more efficiently than 8-byte stores per lane.
+__global__ void __launch_bounds__(kFp8BulkThreads)
+    dispatch_fp8_bulk_kernel(const uint4 *__restrict__ x, int T, int H, int k,
+                             const int32_t *__restrict__ slot_pos, uint8_t *__restrict__ recv_q,
+                             float *__restrict__ recv_scale, long n_rows, int32_t *d_err) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const int in_bytes = 2 * H, q_bytes = H, nb = H >> 7, s_bytes = 4 * nb;
+  unsigned char *in_buf = smem_raw;                                  // [stages][2H]
+  unsigned char *out_q = smem_raw + kFp8BulkStages * in_bytes;       // [H]
+  float *out_s = reinterpret_cast<float *>(out_q + q_bytes);         // [H / 128]
+  __shared__ __align__(8) uint64_t full[kFp8BulkStages];
+  __shared__ int rows[2][EP_MAX_K];
+  __shared__ int timed_out;
+  const int tid = threadIdx.x;
+  const long per_cta = (static_cast<long>(T) + gridDim.x - 1) / gridDim.x;
+  const long first = min(static_cast<long>(T), static_cast<long>(blockIdx.x) * per_cta);
+  const long n_mine = min(static_cast<long>(T), first + per_cta) - first;
+
+  pdl_trigger();
+  if (tid == 0) {
+    for (int s = 0; s < kFp8BulkStages; ++s) mbar_init(&full[s], 1);
+    mbar_init_fence();
+    timed_out = 0;
+  }
+  __syncthreads();
+  pdl_wait();
+
+  auto issue = [&](long i) {  // thread 0: token first + i -> input stage i % stages
+    const int s = static_cast<int>(i % kFp8BulkStages);
+    mbar_arrive_expect_tx(&full[s], in_bytes);
+    bulk_load(in_buf + s * in_bytes, x + (first + i) * (H >> 3), in_bytes, &full[s]);
+  };
+  if (tid == 0)
+    for (long i = 0; i < min(static_cast<long>(kFp8BulkStages - 1), n_mine); ++i) issue(i);
+
+  long i = 0;
+  for (; i < n_mine; ++i) {
+    const long t = first + i;
+    const int s = static_cast<int>(i % kFp8BulkStages);
+    if (tid == 0) {
+      if (i + kFp8BulkStages - 1 < n_mine) issue(i + kFp8BulkStages - 1);
+      bulk_wait_read<0>();  // the previous token's stores have left the output stage
+    }
+    if (tid < k) rows[i & 1][tid] = __ldg(slot_pos + t * k + tid);
+    if (!mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kFp8BulkStages) & 1)))
+      timed_out = 1;
+    __syncthreads();
+    if (timed_out) break;
+    const uint4 *xin = reinterpret_cast<const uint4 *>(in_buf + s * in_bytes);
+    uint2 *qo = reinterpret_cast<uint2 *>(out_q);
+    // 16 consecutive vectors = one block per half-warp; whole warps share
+    // the loop bound because H / 8 is a multiple of 64
+    for (int v = tid; v < (H >> 3); v += kFp8BulkThreads) {
+      float sc;
+      qo[v] = quantize_block_lane(xin[v], &sc);
+      if ((tid & 15) == 0) out_s[v >> 4] = sc;
+    }
+    fence_proxy_async_smem();  // the stage's generic writes before the bulk reads
+    __syncthreads();
+    if (tid == 0) {
+      for (int j = 0; j < k; ++j) {
+        const int row = rows[i & 1][j];
+        if (row < 0 || row >= n_rows) continue;
+        bulk_store(recv_q + static_cast<long>(row) * H, out_q, q_bytes);
+        bulk_store(recv_scale + static_cast<long>(row) * nb, out_s, s_bytes);
+      }
+      bulk_commit();
+    }
+  }
+  if (tid == 0) {
+    if (timed_out) {
+      if (d_err != nullptr) atomicExch(reinterpret_cast<int *>(d_err), EP_ERR_TIMEOUT);
+      for (long q = i + 1; q < min(n_mine, i + kFp8BulkStages); ++q)
+        mbar_wait_bounded(&full[q % kFp8BulkStages],
+                          static_cast<unsigned>((q / kFp8BulkStages) & 1));
+    }
+    bulk_wait<0>();
+  }
+}
+
 // Work item = (token, chunk of 4 blocks of 128 channels).  Lane l covers
 // 8 channels of block 2p + (l >> 4) for p = 0, 1: each half-warp owns a
 // block per load, so the amax reduction is 4 xor-shuffles inside it and
@@ -84,6 +188,8 @@ __global__ void __launch_bounds__(kThreads)
                         const int32_t *__restrict__ slot_pos,
                         uint2 *__restrict__ recv_q,
                         float *__restrict__ recv_scale, long n_rows) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31, half = lane >> 4, sub = lane & 15;
   const int Hv = H >> 3;   // 8-channel units per row (16 B in, 8 B out)
   const int nb = H >> 7;   // 128-channel blocks per row
@@ -155,26 +261,48 @@ cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
   auto kern = dispatch_bf16_kernel<kBf16Vec>;
   const long grid =
       persistent_grid(reinterpret_cast<const void *>(kern), kThreads, 0, items, num_sms);
-  kern<<<grid, kThreads, 0, s>>>(static_cast<const uint4 *>(x), T, Hv, k, slot_pos,
-                                 static_cast<uint4 *>(recv), static_cast<long>(T) * k);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, s, 1, static_cast<const uint4 *>(x), T,
+                    Hv, k, slot_pos, static_cast<uint4 *>(recv), static_cast<long>(T) * k);
 }
+
+// Largest hidden size the bulk FP8 kernel stages in shared memory.
+constexpr int kFp8BulkMaxH = 16384;
+
+int fp8_bulk_smem(int H) { return kFp8BulkStages * 2 * H + H + H / 32; }
 
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
-                                float *recv_scale, int num_sms, int32_t * /*d_err*/,
+                                float *recv_scale, int num_sms, int32_t *d_err,
                                 cudaStream_t s, int *launches) {
+  // bulk stores need 16-byte aligned scale rows: H % 512 == 0 and an
+  // aligned recv_scale
+  if (H % 512 == 0 && H <= kFp8BulkMaxH && reinterpret_cast<uintptr_t>(recv_scale) % 16 == 0) {
+    if (T == 0) return cudaSuccess;
+    const int smem = fp8_bulk_smem(H);
+    const cudaError_t err =
+        raise_dynamic_smem(reinterpret_cast<const void *>(dispatch_fp8_bulk_kernel),
+                           fp8_bulk_smem(kFp8BulkMaxH));
+    if (err != cudaSuccess) return err;
+    const long grid =
+        persistent_grid(reinterpret_cast<const void *>(dispatch_fp8_bulk_kernel),
+                        kFp8BulkThreads, smem, static_cast<long>(T) * (kFp8BulkThreads / kWarp),
+                        num_sms);
+    ++*launches;
+    return launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(kFp8BulkThreads), smem, s, 1,
+                      static_cast<const uint4 *>(x), T, H, k, slot_pos,
+                      static_cast<uint8_t *>(recv_q), recv_scale, static_cast<long>(T) * k,
+                      d_err);
+  }
   const long nchunks = (H / 128 + 3) / 4;
   const long items = static_cast<long>(T) * nchunks;
   if (items == 0) return cudaSuccess;
   const long grid = persistent_grid(reinterpret_cast<const void *>(dispatch_fp8_kernel),
                                     kThreads, 0, items, num_sms);
-  dispatch_fp8_kernel<<<grid, kThreads, 0, s>>>(
-      static_cast<const uint4 *>(x), T, H, k, slot_pos, static_cast<uint2 *>(recv_q),
-      recv_scale, static_cast<long>(T) * k);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(dispatch_fp8_kernel, dim3(grid), dim3(kThreads), 0, s, 1,
+                    static_cast<const uint4 *>(x), T, H, k, slot_pos,
+                    static_cast<uint2 *>(recv_q), recv_scale, static_cast<long>(T) * k);
 }
 
 }  // namespace ep

@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "ep_internal.cuh"
@@ -86,13 +87,14 @@ int device_sm_count() {
 long persistent_grid(const void *kernel, int threads, int smem_bytes, long warp_items,
                      int num_sms) {
   static std::mutex mu;
-  static std::map<std::pair<int, const void *>, int> cache;
+  static std::map<std::tuple<int, const void *, int, int>, int> cache;
   int dev = 0;
   cudaGetDevice(&dev);
   int per_sm = 0;
   {
     std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find({dev, kernel});
+    const auto key = std::make_tuple(dev, kernel, threads, smem_bytes);
+    auto it = cache.find(key);
     if (it != cache.end()) {
       per_sm = it->second;
     } else {
@@ -100,7 +102,7 @@ long persistent_grid(const void *kernel, int threads, int smem_bytes, long warp_
               cudaSuccess ||
           per_sm < 1)
         per_sm = 1;
-      cache[{dev, kernel}] = per_sm;
+      cache[key] = per_sm;
     }
   }
   const int sms = num_sms > 0 ? num_sms : device_sm_count();

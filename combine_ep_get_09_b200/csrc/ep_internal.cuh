@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "ep.h"
 
 namespace ep {
@@ -40,6 +42,19 @@ __device__ __forceinline__ void st_stream_v2(uint2 *p, uint2 v) {
 
 __device__ __forceinline__ void st_stream_f32(float *p, float v) {
   asm volatile("st.global.cs.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+// Programmatic dependent launch (sm_90+).  Every kernel of the library is
+// launched with programmatic stream serialization, so it may be scheduled
+// while the previous kernel on the stream is still running; it must call
+// pdl_wait() before touching memory that kernel writes (griddepcontrol.wait
+// returns once the previous grid has completed and its writes are visible;
+// with no such predecessor it returns at once).  pdl_trigger() lets the
+// next kernel on the stream be scheduled early; that kernel still waits for
+// this one to finish before using its output.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ unsigned lanemask_lt() {
@@ -96,12 +111,39 @@ int device_sm_count();
 // Grid for a persistent kernel: enough blocks of `threads` threads to give
 // each of `warp_items` work items a warp, capped at the blocks that fit at
 // once (with `smem_bytes` of dynamic shared memory each) on `num_sms` SMs
-// (0 = all SMs).  The occupancy figure is cached per (device, kernel).
+// (0 = all SMs).  The occupancy figure is cached per (device, kernel,
+// threads, shared memory).
 long persistent_grid(const void *kernel, int threads, int smem_bytes, long warp_items,
                      int num_sms);
 
 // Raises a kernel's dynamic shared memory limit to `bytes` (once per
 // device and kernel).
 cudaError_t raise_dynamic_smem(const void *kernel, int bytes);
+
+// Launches `kernel` with programmatic stream serialization (see pdl_wait)
+// and, when cluster > 1, a thread-block cluster of that many CTAs.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, int smem,
+                       cudaStream_t stream, int cluster, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace ep

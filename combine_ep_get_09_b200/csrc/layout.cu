@@ -107,22 +107,19 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
   return v;
 }
 
-// Exclusive scan of a[0..n) in shared memory by one warp (each lane owns a
-// contiguous run); returns the total to every lane.
+// Exclusive scan of a[0..n) in shared memory by one warp, 32 consecutive
+// elements per round (conflict-free); returns the total to every lane.
 __device__ int warp_exclusive_scan_smem(int *a, int n) {
   const int lane = threadIdx.x & 31;
-  const int per = (n + 31) / 32;
-  const int beg = min(n, lane * per), end = min(n, beg + per);
-  int local = 0;
-  for (int i = beg; i < end; ++i) local += a[i];
-  const int incl = warp_inclusive_scan(local);
-  int run = incl - local;
-  for (int i = beg; i < end; ++i) {
-    const int c = a[i];
-    a[i] = run;
-    run += c;
+  int carry = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const int x = i < n ? a[i] : 0;
+    const int incl = warp_inclusive_scan(x);
+    if (i < n) a[i] = carry + incl - x;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
   }
-  return __shfl_sync(0xffffffffu, incl, 31);
+  return carry;
 }
 
 // Lanes of the warp whose key equals this lane's, among the lanes in
@@ -195,9 +192,10 @@ __device__ __forceinline__ int rank_one(int e, int bits, int *hist_w) {
 }
 
 template <typename IdT>
-__device__ void rank_segment(const IdT *idx, long beg, long end, int E, int bits,
+__device__ void rank_segment(const IdT *idx, long beg, long end, const Params &p,
                              int32_t *d_err, int *hist_w, int32_t *slot_pos, SegRanks &sr) {
   const int lane = threadIdx.x & 31;
+  const int E = p.E, bits = p.id_bits;
   {
     long long v[kIdBatch];
     load_id_batch(idx, beg, end, v);
@@ -218,7 +216,8 @@ __device__ void rank_segment(const IdT *idx, long beg, long end, int E, int bits
     for (int b = 0; b < kIdBatch; ++b) {
       if (c0 + 32 * b >= end) break;  // uniform across the warp
       const long i = c0 + 32 * b + lane;
-      const int r = rank_one(check_id(v[b], E, d_err), bits, hist_w);
+      const int e = check_id(v[b], E, d_err);
+      const int r = rank_one(e, bits, hist_w);
       if (i < end) slot_pos[i] = r;
     }
   }
@@ -300,24 +299,36 @@ __device__ void rank_mask(const Params &p, int t_beg, int t_end, int *hist_w) {
 
 // ------------------------------------------------------------- cluster path
 
-int cluster_smem_bytes(int E, int R, int warps) {
-  return (warps * (E + R + 1) + 4 * (E + R)) * static_cast<int>(sizeof(int));
+// Split cluster barrier: every thread of every CTA arrives once at kernel
+// start, and waits before its first access to another CTA's shared memory,
+// which is then guaranteed to be running.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
+int cluster_smem_bytes(int E, int R, int warps, int ctas) {
+  return (warps * (E + R + 1) + (ctas + 3) * (E + R)) * static_cast<int>(sizeof(int));
 }
 
 template <typename IdT>
 __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Params p) {
+  pdl_trigger();
   cg::cluster_group cluster = cg::this_cluster();
   const int n_ctas = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
+  if (n_ctas > 1) cluster_arrive_relaxed();
   extern __shared__ int smem[];
   const int E = p.E, R = p.R, C = E + R, ld = hist_ld(p);
   const int tid = threadIdx.x, nt = blockDim.x, w = tid >> 5, nw = nt >> 5;
-  int *hist = smem;            // [warps][E + R + 1]
-  int *mine = hist + nw * ld;  // [C] this CTA's counts, read by all CTAs
-  int *before = mine + C;      // [C] counts of the lower-ranked CTAs
-  int *tot = before + C;       // [C] totals, then exclusive offsets
-  int *base = tot + C;         // [C] first row of each expert for this CTA
-  __shared__ int s_kept;       // rows in use (all CTAs)
+  int *hist = smem;               // [warps][E + R + 1]
+  int *all = hist + nw * ld;      // [ctas][C] every CTA's counts, pushed by each CTA
+  int *before = all + n_ctas * C; // [C] counts of the lower-ranked CTAs
+  int *tot = before + C;          // [C] totals, then exclusive offsets
+  int *base = tot + C;            // [C] first row of each expert for this CTA
+  __shared__ int s_kept;          // rows in use (all CTAs)
   const IdT *idx = static_cast<const IdT *>(p.idx);
 
   const int per_cta = (p.T + n_ctas - 1) / n_ctas;
@@ -328,41 +339,45 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
 
   for (int i = tid; i < nw * ld; i += nt) smem[i] = 0;
   __syncthreads();
+  pdl_wait();
   long seg_end;
   const long seg_beg = warp_slice(n, w, nw, &seg_end);
   SegRanks sr;
-  rank_segment(idx, s_beg + seg_beg, s_beg + seg_end, E, p.id_bits, p.d_err, hist + w * ld,
-               p.slot_pos, sr);
+  rank_segment(idx, s_beg + seg_beg, s_beg + seg_end, p, p.d_err, hist + w * ld, p.slot_pos,
+               sr);
   rank_mask<IdT>(p, t_beg, t_end, hist + w * ld);
   __syncthreads();
-  scan_hist_columns(hist, ld, E, C, nw, mine);  // mine[c] = this CTA's count
-  if (n_ctas > 1) {
-    cluster.sync();  // every CTA's `mine` is complete and visible
-    for (int c = tid; c < C; c += nt) {
-      int b = 0, a = 0;
-      for (int r0 = 0; r0 < n_ctas; r0 += 8) {
-        int v[8];  // 8 remote loads in flight
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          v[u] = r0 + u < n_ctas ? cluster.map_shared_rank(mine, r0 + u)[c] : 0;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          b += r0 + u < rank ? v[u] : 0;
-          a += v[u];
-        }
-      }
-      before[c] = b;
-      tot[c] = a;
+  if (n_ctas > 1) cluster_wait();  // every CTA of the cluster is running
+  // one thread per column: exclusive prefix over this CTA's warps, and the
+  // CTA's count pushed into row `rank` of every CTA's `all`
+  for (int c = tid; c < C; c += nt) {
+    int run = 0;
+    for (int v = 0; v < nw; ++v) {
+      const int x = hist[v * ld + c];
+      if (c < E) hist[v * ld + c] = run;
+      run += x;
     }
-    cluster.sync();  // no CTA reads another's shared memory after this
-  } else {
-    __syncthreads();
-    for (int c = tid; c < C; c += nt) {
-      before[c] = 0;
-      tot[c] = mine[c];
+    if (n_ctas > 1) {
+      for (int q = 0; q < n_ctas; ++q) cluster.map_shared_rank(all, q)[rank * C + c] = run;
+    } else {
+      all[c] = run;
     }
-    __syncthreads();
   }
+  if (n_ctas > 1)
+    cluster.sync();  // all pushes done and visible; nothing remote after this
+  else
+    __syncthreads();
+  for (int c = tid; c < C; c += nt) {
+    int b = 0, a = 0;
+    for (int r = 0; r < n_ctas; ++r) {
+      const int v = all[r * C + c];
+      b += r < rank ? v : 0;
+      a += v;
+    }
+    before[c] = b;
+    tot[c] = a;
+  }
+  __syncthreads();
   if (rank == 0)
     for (int c = tid; c < C; c += nt) {
       if (c < E) p.cnt_e[c] = tot[c];
@@ -403,6 +418,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
 
 template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int smem[];
   const int E = p.E, R = p.R, C = E + R, ld = hist_ld(p);
   const int tid = threadIdx.x, nt = blockDim.x, w = tid >> 5, nw = nt >> 5;
@@ -512,6 +529,8 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
 
 template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads) layout_place_kernel(Params p) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int smem[];
   const int E = p.E, C = p.E + p.R, ld = hist_ld(p);
   const int tid = threadIdx.x, w = tid >> 5;
@@ -532,8 +551,8 @@ __global__ void __launch_bounds__(kTileThreads) layout_place_kernel(Params p) {
   long seg_end;
   const long seg_beg = warp_slice(n, w, kTileWarps, &seg_end);
   SegRanks sr;
-  rank_segment(idx, s_beg + seg_beg, s_beg + seg_end, E, p.id_bits, nullptr, hist + w * ld,
-               p.slot_pos, sr);
+  rank_segment(idx, s_beg + seg_beg, s_beg + seg_end, p, nullptr, hist + w * ld, p.slot_pos,
+               sr);
   __syncthreads();
   scan_hist_columns(hist, ld, E, E, kTileWarps, scratch);
   __syncthreads();
@@ -599,32 +618,19 @@ cudaError_t launch_cluster(Params p, cudaStream_t s, int *launches) {
   auto kern = layout_cluster_kernel<IdT>;
   const long N = static_cast<long>(p.T) * p.k;
   const int threads = N <= kSmallSlots ? kSmallThreads : kClusterThreads;
-  const int smem = cluster_smem_bytes(p.E, p.R, threads / kWarp);
-  cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern),
-                                       cluster_smem_bytes(p.E, p.R, kClusterWarps));
+  cudaError_t err = raise_dynamic_smem(
+      reinterpret_cast<const void *>(kern),
+      cluster_smem_bytes(p.E, p.R, kClusterWarps, kMaxClusterCtas));
   if (err != cudaSuccess) return err;
   long want = (N + kSlotsPerClusterCta - 1) / kSlotsPerClusterCta;
   if (want < 1) want = 1;
-  const int cap = want > 8 ? max_cluster_ctas<IdT>(smem) : 8;
+  const int cap = want > 8 ? max_cluster_ctas<IdT>(cluster_smem_bytes(
+                                 p.E, p.R, threads / kWarp, kMaxClusterCtas))
+                           : 8;
   const int n_ctas = static_cast<int>(want < cap ? want : cap);
+  const int smem = cluster_smem_bytes(p.E, p.R, threads / kWarp, n_ctas);
   ++*launches;
-  if (n_ctas == 1) {  // a plain launch: the kernel sees a cluster of one
-    kern<<<1, threads, smem, s>>>(p);
-    return cudaGetLastError();
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_ctas);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = n_ctas;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return launch_pdl(kern, dim3(n_ctas), dim3(threads), smem, s, n_ctas, p);
 }
 
 template <typename IdT>
@@ -638,13 +644,13 @@ cudaError_t launch_tiled(Params p, cudaStream_t s, int *launches) {
   if (err != cudaSuccess) return err;
   err = raise_dynamic_smem(reinterpret_cast<const void *>(layout_place_kernel<IdT>), place_smem);
   if (err != cudaSuccess) return err;
-  layout_count_kernel<IdT><<<p.ntiles, kTileThreads, count_smem, s>>>(p);
   ++*launches;
-  err = cudaGetLastError();
+  err = launch_pdl(layout_count_kernel<IdT>, dim3(p.ntiles), dim3(kTileThreads), count_smem, s,
+                   1, p);
   if (err != cudaSuccess) return err;
-  layout_place_kernel<IdT><<<p.ntiles, kTileThreads, place_smem, s>>>(p);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(layout_place_kernel<IdT>, dim3(p.ntiles), dim3(kTileThreads), place_smem,
+                    s, 1, p);
 }
 
 }  // namespace

@@ -192,10 +192,27 @@ def test_dispatch_fp8_full_size(name):
     _dispatch_fp8_check(cfg, b)
 
 
-@pytest.mark.parametrize("H", [128, 256, 384, 640, 896, 7168, 7296])
+@pytest.mark.parametrize("H", [128, 256, 384, 512, 640, 896, 1536, 4096, 7168, 7296, 16384])
 def test_dispatch_fp8_ragged_hidden(H):
+    # H % 512 == 0 (up to 16384) takes the shared-memory bulk-copy kernel,
+    # other multiples of 128 the register kernel
     cfg, b = _batch("decode", 7, T=77, H=H, drop_frac=0.1)
     _dispatch_fp8_check(cfg, b)
+
+
+def test_dispatch_fp8_misaligned_scales_use_register_path():
+    # scale rows 4-byte (not 16-byte) aligned: bulk stores are not allowed
+    cfg, b = _batch("decode", 13, T=50, H=1024)
+    T, H, k = b.T, b.H, cfg.k
+    L, g = gpu_layout(b.idx, cfg.E, cfg.R)
+    ref = oracle.layout(b.idx, cfg.E, cfg.R)
+    q = torch.full((T * k, H), CANARY8, dtype=torch.uint8, device="cuda")
+    s_buf = torch.full((T * k * (H // 128) + 1,), -1.0, dtype=torch.float32, device="cuda")
+    s = s_buf[1:].view(T * k, H // 128)             # offset by 4 bytes
+    ep.ep_dispatch(b.x.cuda(), L.slot_pos, fp8=True, recv=q, recv_scale=s)
+    wq, ws_ = oracle.dispatch_fp8(b.x, ref["slot_pos"], T * k)
+    np.testing.assert_array_equal(tensor_bytes(q), wq)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), ws_.view(np.uint32))
 
 
 def test_dispatch_fp8_special_values():
