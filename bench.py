@@ -349,6 +349,8 @@ def bench_ours(args, world, rank, device):
     }
     if not args.skip_decode:
         result["decode"] = bench_decode(ep, device, world)
+    if not args.skip_dedup:
+        result["rank_dedup"] = bench_rank_dedup(ep, st, cfg, device, world)
     if not args.skip_e2e:
         result["e2e"] = bench_e2e(ep, cfg, batch, device, args, world, total_bytes)
     if world == 1 and rank == 0 and not args.skip_cpu:
@@ -391,6 +393,58 @@ def profiled_traffic(kernel: str):
     if not m or not t or m.group(1) != kernel_source_digest(kernel):
         return None
     return float(t.group(1))
+
+
+def bench_rank_dedup(ep, st, cfg, device, world, iters=20):
+    """The rank-deduplicated path on the same prefill batch: rank rows from
+    the token-in-rank mask, dispatch into one row per (token, rank), and the
+    unit-weight combine of per-rank partial outputs.  Each kernel is timed
+    alone (flushed L2) and reported with its algorithmic bytes."""
+    T, H, R = cfg.T, cfg.H, cfg.R
+    stream = torch.cuda.Stream(device)
+    flush = L2Flush(device)
+    with torch.cuda.stream(stream):
+        st.run(stream)
+        rl = ep.ep_get_rank_layout(st.layout.in_rank, stream=stream)
+    stream.synchronize()
+    rows = int(rl.off_r[-1].item())
+    recv = torch.empty((T * R, H), dtype=torch.bfloat16, device=device)
+    q = torch.empty((T * R, H), dtype=torch.float8_e4m3fn, device=device)
+    sc = torch.empty((T * R, H // 128), dtype=torch.float32, device=device)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    calls = {
+        "rank_layout": (lambda: ep.ep_get_rank_layout(st.layout.in_rank, out=rl, stream=stream),
+                        T * R + (2 * R + 1) * 4 + 2 * T * R * 4),
+        "dispatch_bf16": (lambda: ep.ep_dispatch(st.x, rl.rank_row, recv=recv, stream=stream),
+                          T * H * 2 + rows * H * 2),
+        "dispatch_fp8": (lambda: ep.ep_dispatch(st.x, rl.rank_row, fp8=True, recv=q,
+                                                recv_scale=sc, stream=stream),
+                         T * H * 2 + rows * (H + H // 32)),
+        "combine": (lambda: ep.ep_combine(recv, rl.rank_row, None, out=out, stream=stream),
+                    rows * H * 2 + T * H * 2),
+    }
+    res = {"rows": rows, "expert_rows": T * cfg.k,
+           "write_saving": round(1 - rows / (T * cfg.k), 4)}
+    for name, (fn, nbytes) in calls.items():
+        evs = []
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                flush()
+                fn()
+            for _ in range(iters):
+                flush()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                evs.append((a, b))
+        stream.synchronize()
+        us = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3,
+                            world, device)
+        res[name] = {"us": round(us, 2), "bytes": nbytes,
+                     "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)}
+    return res
 
 
 def bench_decode(ep, device, world, iters=200):
@@ -624,6 +678,7 @@ def main():
     p.add_argument("--skip-decode", action="store_true")
     p.add_argument("--skip-e2e", action="store_true")
     p.add_argument("--skip-cpu", action="store_true")
+    p.add_argument("--skip-dedup", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--reference-tokens", type=int, default=256)
     p.add_argument("--profile", choices=("layout", "dispatch_bf16", "dispatch_fp8", "combine"),

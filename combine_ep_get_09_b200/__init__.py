@@ -19,7 +19,8 @@ from typing import NamedTuple, Optional
 
 import torch
 
-__all__ = ["EPError", "EPLibraryError", "Layout", "ep_get_layout",
+__all__ = ["EPError", "EPLibraryError", "Layout", "RankLayout", "ep_get_layout",
+           "ep_get_rank_layout", "ep_rank_layout_workspace_bytes",
            "ep_get_layout_noalloc", "EP_NOALLOC_SCRATCH_BYTES",
            "ep_dispatch", "ep_combine", "ep_read_error",
            "ep_layout_workspace_bytes", "ep_kernel_launches", "lib",
@@ -65,6 +66,8 @@ _SIGNATURES = {
     "ep_read_error": ([_vp, _vp], _i),
     "ep_get_layout_noalloc": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                _vp, _vp, _vp, _vp], _i),
+    "ep_rank_layout_workspace_bytes": ([_i, _i], _sz),
+    "ep_get_rank_layout": ([_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i),
 }
 
 
@@ -185,6 +188,42 @@ def ep_get_layout_noalloc(idx: torch.Tensor, E: int, R: int, *,
     return out
 
 
+class RankLayout(NamedTuple):
+    cnt_r: torch.Tensor     # [R] int32
+    off_r: torch.Tensor     # [R+1] int32
+    rank_row: torch.Tensor  # [T, R] int32
+    rank_src: torch.Tensor  # [T*R] int32
+
+
+def ep_rank_layout_workspace_bytes(T: int, R: int) -> int:
+    return int(lib().ep_rank_layout_workspace_bytes(T, R))
+
+
+def ep_get_rank_layout(in_rank: torch.Tensor, *, out: Optional[RankLayout] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> RankLayout:
+    """Rows of the rank-deduplicated dispatch from the token-in-rank mask
+    ``in_rank`` [T, R] (uint8) of ep_get_layout: one row per (token, rank)
+    pair.  Dispatch with ``ep_dispatch(x, rank_row)``; combine per-rank
+    partial outputs with ``ep_combine(z, rank_row, None)``."""
+    _need_cuda("in_rank", in_rank)
+    if in_rank.dtype != torch.uint8 or in_rank.dim() != 2:
+        raise ValueError("in_rank must be a 2-D uint8 tensor")
+    T, R = in_rank.shape
+    dev = in_rank.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = RankLayout(torch.empty(R, **i32), torch.empty(R + 1, **i32),
+                         torch.empty((T, R), **i32), torch.empty(T * R, **i32))
+    need = ep_rank_layout_workspace_bytes(T, R)
+    if ws is None and need > 0:
+        ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    _check(lib().ep_get_rank_layout(
+        _ptr(in_rank), T, R, _ptr(out.cnt_r), _ptr(out.off_r), _ptr(out.rank_row),
+        _ptr(out.rank_src), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _stream(stream)))
+    return out
+
+
 def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
                 recv: Optional[torch.Tensor] = None,
                 recv_scale: Optional[torch.Tensor] = None,
@@ -211,15 +250,18 @@ def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
     return (recv, recv_scale) if fp8 else recv
 
 
-def ep_combine(y: torch.Tensor, slot_pos: torch.Tensor, w: torch.Tensor, *,
+def ep_combine(y: torch.Tensor, slot_pos: torch.Tensor, w: Optional[torch.Tensor], *,
                out: Optional[torch.Tensor] = None, num_sms: int = 0,
                d_err: Optional[torch.Tensor] = None,
                stream=None) -> torch.Tensor:
     """Gate-weighted combine of expert outputs ``y`` [T*k, H] bf16 into
-    ``out`` [T, H] bf16 (fp32 fma chain in slot order)."""
-    for name, t in (("y", y), ("slot_pos", slot_pos), ("w", w)):
+    ``out`` [T, H] bf16 (fp32 fma chain in slot order).  ``w=None`` sums
+    the slot rows with unit weights."""
+    for name, t in (("y", y), ("slot_pos", slot_pos)):
         _need_cuda(name, t)
-    if y.dtype != torch.bfloat16 or w.dtype != torch.float32:
+    if w is not None:
+        _need_cuda("w", w)
+    if y.dtype != torch.bfloat16 or (w is not None and w.dtype != torch.float32):
         raise ValueError("y must be bf16 and w fp32")
     T, k = slot_pos.shape
     H = y.shape[1]

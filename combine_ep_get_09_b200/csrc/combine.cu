@@ -1,5 +1,7 @@
 // combine.cu -- gate-weighted sum of the expert outputs back into token
-// order: out[t] = bf16(fma chain over slots j = 0..k-1 of w[t,j] * y[row]).
+// order: out[t] = bf16(fma chain over slots j = 0..k-1 of w[t,j] * y[row]),
+// every w[t,j] = 1 when no weights are given (a plain sum, as combining
+// per-rank partial outputs needs).
 //
 // Two kernels, both fp32 fma chains in slot order (so both bit-identical):
 //
@@ -90,7 +92,7 @@ __global__ void __launch_bounds__(kChunkVec)
       float wj = 0.0f;
       if (j < k) {
         r = __ldg(slot_pos + static_cast<long>(t) * k + j);
-        wj = __ldg(w + static_cast<long>(t) * k + j);
+        wj = w != nullptr ? __ldg(w + static_cast<long>(t) * k + j) : 1.0f;
         if (r < 0 || r >= n_rows) r = -1;
       }
       rows[j] = r;
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(kRegThreads, 2)
     const int c = static_cast<int>(it - static_cast<long>(t) * nchunks);
     const long tk = static_cast<long>(t) * k;
     const int sp = lane < k ? __ldg(slot_pos + tk + lane) : -1;
-    const float wt = lane < k ? __ldg(w + tk + lane) : 0.0f;
+    const float wt = lane < k ? (w != nullptr ? __ldg(w + tk + lane) : 1.0f) : 0.0f;
     const int v = c * 32 + lane;
 
     float acc[8];

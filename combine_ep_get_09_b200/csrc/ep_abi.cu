@@ -186,7 +186,7 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
   }
   ep::LayoutArgs a{};
   a.idx = idx;
-  a.idx_is_int64 = idx_is_int64 ? 1 : 0;
+  a.id_kind = idx_is_int64 ? ep::kIdsInt64 : ep::kIdsInt32;
   a.T = T;
   a.k = k;
   a.E = E;
@@ -200,6 +200,54 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
   a.in_rank = in_rank;
   a.ws = ws;
   a.d_err = d_err;
+  int n = 0;
+  const cudaError_t e = ep::launch_layout(a, static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
+  return from_cuda(e, fn);
+}
+
+size_t ep_rank_layout_workspace_bytes(int T, int R) {
+  if (T < 0 || R < 1 || R > EP_MAX_R || static_cast<long long>(T) * R > 0x7fffffffLL) return 0;
+  return ep::layout_workspace_bytes(T, R, R, 1);
+}
+
+ep_status_t ep_get_rank_layout(const uint8_t *in_rank, int T, int R, int32_t *cnt_r,
+                               int32_t *off_r, int32_t *rank_row, int32_t *rank_src,
+                               void *ws, size_t ws_bytes, void *stream) {
+  static const char fn[] = "ep_get_rank_layout";
+  g_err[0] = '\0';
+  if (T < 0) return fail(EP_ERR_INVALID_ARG, "%s: T=%d < 0", fn, T);
+  if (R < 1) return fail(EP_ERR_INVALID_ARG, "%s: R=%d < 1", fn, R);
+  if (R > EP_MAX_R) return fail(EP_ERR_UNSUPPORTED, "%s: R=%d > %d", fn, R, EP_MAX_R);
+  if (static_cast<long long>(T) * R > 0x7fffffffLL)
+    return fail(EP_ERR_UNSUPPORTED, "%s: T*R does not fit int32", fn);
+  EP_REQUIRE_PTR(fn, cnt_r, 4);
+  EP_REQUIRE_PTR(fn, off_r, 4);
+  if (T > 0) {
+    EP_REQUIRE_PTR(fn, in_rank, 1);
+    EP_REQUIRE_PTR(fn, rank_row, 4);
+    EP_REQUIRE_PTR(fn, rank_src, 4);
+  }
+  const size_t need = ep::layout_workspace_bytes(T, R, R, 1);
+  if (need > 0) {
+    EP_REQUIRE_PTR(fn, ws, 16);
+    if (ws_bytes < need)
+      return fail(EP_ERR_INVALID_ARG, "%s: ws_bytes=%zu < %zu needed", fn, ws_bytes, need);
+  }
+  // the expert layout of the mask: slot (t, r) "chooses expert r" when token
+  // t is in rank r; experts = ranks, one group holding them all
+  ep::LayoutArgs a{};
+  a.idx = in_rank;
+  a.id_kind = ep::kIdsMask;
+  a.T = T;
+  a.k = R;
+  a.E = R;
+  a.R = 1;
+  a.cnt_e = cnt_r;
+  a.off_e = off_r;
+  a.slot_pos = rank_row;
+  a.recv_src = rank_src;
+  a.ws = ws;
   int n = 0;
   const cudaError_t e = ep::launch_layout(a, static_cast<cudaStream_t>(stream), &n);
   g_launches += n;
@@ -241,7 +289,8 @@ ep_status_t ep_combine(const void *y, int T, int H, int k,
   if (T == 0) return EP_OK;
   EP_REQUIRE_PTR(fn, y, 16);
   EP_REQUIRE_PTR(fn, slot_pos, 4);
-  EP_REQUIRE_PTR(fn, w, 4);
+  if (w != nullptr && !aligned(w, 4))
+    return fail(EP_ERR_INVALID_ARG, "%s: w is not 4-byte aligned", fn);
   EP_REQUIRE_PTR(fn, out, 16);
   if (d_err != nullptr && !aligned(d_err, 4))
     return fail(EP_ERR_INVALID_ARG, "%s: d_err is not 4-byte aligned", fn);

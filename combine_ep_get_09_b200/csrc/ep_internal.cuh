@@ -67,9 +67,14 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // Each returns cudaSuccess or the launch error; arguments are validated by
 // the ABI layer before these are called.
 
+// What LayoutArgs::idx points at.
+constexpr int kIdsInt32 = 0;  // int32 expert ids [T, k]
+constexpr int kIdsInt64 = 1;  // int64 expert ids [T, k]
+constexpr int kIdsMask = 2;   // uint8 mask [T, k]: slot (t, j) is expert j when set
+
 struct LayoutArgs {
   const void *idx;
-  int idx_is_int64;
+  int id_kind;
   int T, k, E, R;
   int32_t *cnt_e, *cnt_r, *off_e, *off_r, *slot_pos, *recv_src;
   uint8_t *in_rank;

@@ -74,18 +74,31 @@ __device__ __forceinline__ int rank_of(int e, const Params &p) {
   return static_cast<int>((static_cast<unsigned long long>(e) * p.g_magic) >> 32);
 }
 
+// Raw id of flat slot i.  int64 / int32 ids are read as they are; a uint8
+// token-in-rank mask [T, k] is read as "slot (t, r) belongs to expert r"
+// (r = i % k) when set, else dropped -- the rank-row layout is the expert
+// layout of that mask.
+template <typename IdT>
+__device__ __forceinline__ long long raw_id(const IdT *idx, long i, int /*k*/) {
+  return static_cast<long long>(idx[i]);
+}
+template <>
+__device__ __forceinline__ long long raw_id<uint8_t>(const uint8_t *idx, long i, int k) {
+  return idx[i] ? static_cast<long long>(i % k) : -1;
+}
+
 // Ids are read kIdBatch at a time per lane, all loads issued before any is
 // used, so a warp pays one memory round trip per kIdBatch * 32 slots.
 constexpr int kIdBatch = 8;
 
 template <typename IdT>
-__device__ __forceinline__ void load_id_batch(const IdT *idx, long c0, long end,
+__device__ __forceinline__ void load_id_batch(const IdT *idx, long c0, long end, int k,
                                               long long (&v)[kIdBatch]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int b = 0; b < kIdBatch; ++b) {
     const long i = c0 + 32 * b + lane;
-    v[b] = i < end ? static_cast<long long>(idx[i]) : -1;
+    v[b] = i < end ? raw_id(idx, i, k) : -1;
   }
 }
 
@@ -198,7 +211,7 @@ __device__ void rank_segment(const IdT *idx, long beg, long end, const Params &p
   const int E = p.E, bits = p.id_bits;
   {
     long long v[kIdBatch];
-    load_id_batch(idx, beg, end, v);
+    load_id_batch(idx, beg, end, p.k, v);
 #pragma unroll
     for (int b = 0; b < kRegChunks; ++b) {
       sr.packed[b] = -1;
@@ -211,7 +224,7 @@ __device__ void rank_segment(const IdT *idx, long beg, long end, const Params &p
   }
   for (long c0 = beg + 32 * kRegChunks; c0 < end; c0 += 32 * kIdBatch) {
     long long v[kIdBatch];
-    load_id_batch(idx, c0, end, v);
+    load_id_batch(idx, c0, end, p.k, v);
 #pragma unroll
     for (int b = 0; b < kIdBatch; ++b) {
       if (c0 + 32 * b >= end) break;  // uniform across the warp
@@ -240,7 +253,7 @@ __device__ void place_segment(const IdT *idx, long beg, long end, int k, int E,
   }
   for (long c0 = beg + 32 * kRegChunks; c0 < end; c0 += 32 * kIdBatch) {
     long long v[kIdBatch];
-    load_id_batch(idx, c0, end, v);
+    load_id_batch(idx, c0, end, k, v);
 #pragma unroll
     for (int b = 0; b < kIdBatch; ++b) {
       const long i = c0 + 32 * b + lane;
@@ -271,7 +284,7 @@ __device__ void rank_mask(const Params &p, int t_beg, int t_end, int *hist_w) {
         long long v[kIdBatch];
 #pragma unroll
         for (int b = 0; b < kIdBatch; ++b)
-          v[b] = j0 + b < p.k ? static_cast<long long>(idx[base + j0 + b]) : -1;
+          v[b] = j0 + b < p.k ? raw_id(idx, base + j0 + b, p.k) : -1;
 #pragma unroll
         for (int b = 0; b < kIdBatch; ++b) {
           const int e = check_id(v[b], p.E, nullptr);
@@ -279,7 +292,9 @@ __device__ void rank_mask(const Params &p, int t_beg, int t_end, int *hist_w) {
         }
       }
       uint8_t *row = p.in_rank + static_cast<long>(t) * p.R;
-      if ((p.R & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 3) == 0) {
+      if (p.in_rank == nullptr) {
+        // mask layouts have no rank rows to write
+      } else if ((p.R & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 3) == 0) {
         // 4 mask bytes per 32-bit store
         for (int r = 0; r < p.R; r += 4) {
           const unsigned b = static_cast<unsigned>(m >> r);
@@ -381,7 +396,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
   if (rank == 0)
     for (int c = tid; c < C; c += nt) {
       if (c < E) p.cnt_e[c] = tot[c];
-      else p.cnt_r[c - E] = tot[c];
+      else if (p.cnt_r != nullptr) p.cnt_r[c - E] = tot[c];
     }
   // warp 0 scans the expert totals, warp 1 the rank totals
   if (w == 0) {
@@ -392,13 +407,13 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
     }
   } else if (w == 1) {
     const int n_tok = warp_exclusive_scan_smem(tot + E, R);
-    if (rank == 0 && (tid & 31) == 0) p.off_r[R] = n_tok;
+    if (rank == 0 && (tid & 31) == 0 && p.off_r != nullptr) p.off_r[R] = n_tok;
   }
   __syncthreads();
   for (int c = tid; c < C; c += nt) {
     if (rank == 0) {
       if (c < E) p.off_e[c] = tot[c];
-      else p.off_r[c - E] = tot[c];
+      else if (p.off_r != nullptr) p.off_r[c - E] = tot[c];
     }
     if (c < E) base[c] = tot[c] + before[c];
   }
@@ -441,7 +456,7 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
 #pragma unroll
     for (int b = 0; b < kIdBatch; ++b) {
       const long i = c0 + static_cast<long>(b) * nt + tid;
-      v[b] = i < s_end ? static_cast<long long>(idx[i]) : -1;
+      v[b] = i < s_end ? raw_id(idx, i, p.k) : -1;
     }
 #pragma unroll
     for (int b = 0; b < kIdBatch; ++b) {
@@ -490,7 +505,7 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
     for (int pp = 0; pp < P; ++pp) s += part[pp * C + c];
     col[c] = s;
     if (c < E) p.cnt_e[c] = s;
-    else p.cnt_r[c - E] = s;
+    else if (p.cnt_r != nullptr) p.cnt_r[c - E] = s;
   }
   __syncthreads();
   if (w == 0) {
@@ -498,12 +513,12 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
     if (tid == 0) p.off_e[E] = n_kept;
   } else if (w == 1) {
     const int n_tok = warp_exclusive_scan_smem(col + E, R);
-    if ((tid & 31) == 0) p.off_r[R] = n_tok;
+    if ((tid & 31) == 0 && p.off_r != nullptr) p.off_r[R] = n_tok;
   }
   __syncthreads();
   for (int c = tid; c < C; c += nt) {
     if (c < E) p.off_e[c] = col[c];
-    else p.off_r[c - E] = col[c];
+    else if (p.off_r != nullptr) p.off_r[c - E] = col[c];
   }
   // absolute row base of every (tile, expert), in place
   for (int q = tid; q < C * P; q += nt) {
@@ -681,15 +696,18 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s, int *launches) {
   p.recv_src = a.recv_src;
   p.in_rank = a.in_rank;
   p.d_err = a.d_err;
-  if (cluster_path(a.T, a.k))
-    return a.idx_is_int64 ? launch_cluster<int64_t>(p, s, launches)
-                          : launch_cluster<int32_t>(p, s, launches);
+  if (cluster_path(a.T, a.k)) {
+    if (a.id_kind == kIdsMask) return launch_cluster<uint8_t>(p, s, launches);
+    return a.id_kind == kIdsInt64 ? launch_cluster<int64_t>(p, s, launches)
+                                  : launch_cluster<int32_t>(p, s, launches);
+  }
   p.tile_T = tile_tokens(a.T);
   p.ntiles = (a.T + p.tile_T - 1) / p.tile_T;
   p.ticket = static_cast<unsigned *>(a.ws);
   p.cols = reinterpret_cast<int32_t *>(static_cast<char *>(a.ws) + kTicketBytes);
-  return a.idx_is_int64 ? launch_tiled<int64_t>(p, s, launches)
-                        : launch_tiled<int32_t>(p, s, launches);
+  if (a.id_kind == kIdsMask) return launch_tiled<uint8_t>(p, s, launches);
+  return a.id_kind == kIdsInt64 ? launch_tiled<int64_t>(p, s, launches)
+                                : launch_tiled<int32_t>(p, s, launches);
 }
 
 }  // namespace ep

@@ -157,13 +157,49 @@ ep_status_t ep_dispatch(const void *x, int T, int H, int k,
  *   out[t, :] = bf16 round-to-nearest-even(acc)
  * y          [T*k, H] bf16 expert outputs in receive-row order.
  * slot_pos   [T,k] int32; values outside [0, T*k) are skipped.
- * w          [T,k] fp32 gate weights (4-byte aligned).
+ * w          [T,k] fp32 gate weights (4-byte aligned), or NULL for unit
+ *            weights: out[t] is then the plain fp32 sum of the kept slot
+ *            rows (how per-rank partial outputs combine, see
+ *            ep_get_rank_layout).
  * out        [T,H] bf16; a token with no kept slot gets +0.
  * Limits as ep_dispatch (H % 8 == 0).  num_sms and d_err as ep_dispatch.
  */
 ep_status_t ep_combine(const void *y, int T, int H, int k,
                        const int32_t *slot_pos, const float *w, void *out,
                        int num_sms, int32_t *d_err, void *stream);
+
+/*
+ * ep_get_rank_layout -- rows of the rank-deduplicated dispatch: one receive
+ * row per (token, rank) pair instead of one per (token, expert).
+ *
+ * DeepEP's high-throughput ("normal") kernels send a token once to each
+ * peer rank that hosts any of its experts (frogred8 blog, "Implementation
+ * of SMs dedicated to network communication": one sender per NVLink peer;
+ * chinainews.com item, "Technical Details": normal kernels for training
+ * and prefill over NVLink and RDMA); the receiving rank then spreads it
+ * over its local experts.  Here, from the token-in-rank mask of
+ * ep_get_layout:
+ *   rank_row[t,r] = off_r[r] + #{t' < t : in_rank[t',r]}  if in_rank[t,r],
+ *                   else -1 (rows of one rank in ascending token order)
+ *   rank_src[q]   = token of rank row q; -1 past off_r[R]
+ *   cnt_r, off_r  = tokens per rank and their exclusive scan (the same
+ *                   values ep_get_layout writes)
+ * Rows per token drop from k to the number of distinct ranks among its
+ * experts (at most min(k, R)).  The dispatch itself is ep_dispatch with
+ * slot_pos = rank_row and k = R (R <= EP_MAX_K there); the matching combine
+ * is ep_combine with slot_pos = rank_row, k = R and w = NULL, summing the
+ * per-rank partial outputs (each already gate-weighted on its rank).
+ *
+ * in_rank   [T,R] uint8 (0 / nonzero), rank_row [T,R] int32,
+ * rank_src  [T*R] int32, cnt_r [R], off_r [R+1] int32.
+ * T >= 0, 1 <= R <= EP_MAX_R, T*R < 2^31.  ws / ws_bytes as ep_get_layout,
+ * sized by ep_rank_layout_workspace_bytes (0 for T*R <= 2^19).
+ */
+size_t ep_rank_layout_workspace_bytes(int T, int R);
+ep_status_t ep_get_rank_layout(const uint8_t *in_rank, int T, int R,
+                               int32_t *cnt_r, int32_t *off_r,
+                               int32_t *rank_row, int32_t *rank_src, void *ws,
+                               size_t ws_bytes, void *stream);
 
 /* Size of the scratch array behind ep_get_layout_noalloc (256 KiB). */
 #define EP_NOALLOC_SCRATCH_BYTES (256u * 1024u)

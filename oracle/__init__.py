@@ -49,6 +49,9 @@ def lib():
             _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             _i32p, _i32p, _u8p, _i32p, _i32p, _i32p, _i32p]
         L.ep_oracle_layout.restype = ctypes.c_int
+        L.ep_oracle_rank_layout.argtypes = [_u8p, ctypes.c_int, ctypes.c_int, _i32p, _i32p,
+                                            _i32p, _i32p]
+        L.ep_oracle_rank_layout.restype = ctypes.c_int
         L.ep_oracle_dispatch_bf16.argtypes = [
             _u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i32p,
             ctypes.c_long, _u16p]
@@ -153,6 +156,21 @@ def layout(idx, E: int, R: int) -> Dict[str, np.ndarray]:
     return out
 
 
+def rank_layout(in_rank) -> Dict[str, np.ndarray]:
+    """Rank rows of the token-in-rank mask in_rank [T, R] (uint8):
+    cnt_r[R], off_r[R+1], rank_row[T, R], rank_src[T*R]."""
+    m = np.ascontiguousarray(_np(in_rank, np.uint8))
+    T, R = m.shape
+    out = dict(cnt_r=np.zeros(R, np.int32), off_r=np.zeros(R + 1, np.int32),
+               rank_row=np.zeros((T, R), np.int32), rank_src=np.zeros(T * R, np.int32))
+    st = lib().ep_oracle_rank_layout(_ptr(m, _u8p), T, R, _ptr(out["cnt_r"], _i32p),
+                                     _ptr(out["off_r"], _i32p), _ptr(out["rank_row"], _i32p),
+                                     _ptr(out["rank_src"], _i32p))
+    if st:
+        raise ValueError("oracle rank_layout: invalid arguments")
+    return out
+
+
 # ----------------------------------------------------------------- dispatch
 
 def dispatch_bf16(x, slot_pos, n_rows: int, recv: np.ndarray = None) -> np.ndarray:
@@ -198,10 +216,10 @@ def dispatch_fp8(x, slot_pos, n_rows: int, recv_q: np.ndarray = None,
 
 def combine(y, slot_pos, w) -> np.ndarray:
     """out[t] = bf16(fma chain over slots of w[t, j] * y[slot_pos[t, j]]),
-    as uint16 bf16 bits [T, H]."""
+    as uint16 bf16 bits [T, H]; w=None means every weight is 1."""
     yb = _np(y, np.uint16)
     sp = _np(slot_pos, np.int32)
-    wf = _np(w, np.float32)
+    wf = np.ones(sp.shape, np.float32) if w is None else _np(w, np.float32)
     n_rows, H = yb.shape
     T, k = sp.shape
     out = np.zeros((T, H), np.uint16)

@@ -34,6 +34,12 @@
  *   combine  out[t,:] = bf16_rne( fma chain over j = 0..k-1 in slot order of
  *                       w[t,j] * y[slot_pos[t,j], :], starting from 0.0f )
  *
+ *   rank layout (the rank-deduplicated form of dispatch: one row per
+ *            (token, rank) pair, DeepEP's per-peer sends)
+ *            rank_row[t,r] = off_r[r] + #{t' < t : in_rank[t',r]} if
+ *                            in_rank[t,r], else -1
+ *            rank_src[q]   = token of rank row q (-1 past the last)
+ *
  * Slots with idx == -1 are dropped: slot_pos = -1, nothing is written for
  * them and combine skips them.  An id outside [-1, E) is reported
  * (return value EP_ORACLE_ERR_INDEX) and treated like a dropped slot.
@@ -206,6 +212,42 @@ int ep_oracle_layout(const int64_t *idx, int T, int k, int E, int R,
     for (int r = 0; r < R; ++r)
         off_r[r + 1] = off_r[r] + cnt_r[r];
     return status;
+}
+
+/* Rank rows from the token-in-rank mask in_rank[T,R]: walk tokens in order,
+ * handing each (token, rank) pair the next free row of its rank. */
+int ep_oracle_rank_layout(const uint8_t *in_rank, int T, int R, int32_t *cnt_r,
+                          int32_t *off_r, int32_t *rank_row, int32_t *rank_src) {
+    if (T < 0 || R <= 0)
+        return EP_ORACLE_ERR_INVALID_ARG;
+    for (int r = 0; r < R; ++r)
+        cnt_r[r] = 0;
+    for (long i = 0; i < (long)T * R; ++i)
+        if (in_rank[i])
+            cnt_r[i % R] += 1;
+    off_r[0] = 0;
+    for (int r = 0; r < R; ++r)
+        off_r[r + 1] = off_r[r] + cnt_r[r];
+    int32_t *next = (int32_t *)malloc(sizeof(int32_t) * (size_t)R);
+    if (!next)
+        return EP_ORACLE_ERR_INVALID_ARG;
+    for (int r = 0; r < R; ++r)
+        next[r] = off_r[r];
+    for (long q = 0; q < (long)T * R; ++q)
+        rank_src[q] = -1;
+    for (int t = 0; t < T; ++t) {
+        for (int r = 0; r < R; ++r) {
+            const long i = (long)t * R + r;
+            if (!in_rank[i]) {
+                rank_row[i] = -1;
+                continue;
+            }
+            rank_row[i] = next[r]++;
+            rank_src[rank_row[i]] = t;
+        }
+    }
+    free(next);
+    return EP_ORACLE_OK;
 }
 
 /* --------------------------------------------------------------- dispatch */

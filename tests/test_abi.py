@@ -103,7 +103,7 @@ def test_dispatch_combine_empty_batch_is_a_no_op():
 
 
 @pytest.mark.parametrize("args,status", [
-    ((16, 4, 64, 2, 16, None, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),  # no w
+    ((None, 4, 64, 2, 16, None, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),  # no y
     ((16, 4, 64, 2, 16, 18, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),    # w misaligned
     ((16, 4, 60, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_UNSUPPORTED),
     ((16, 4, 64, 2, 16, 16, 40, 0, None, None), ep.EP_ERR_INVALID_ARG),    # out misaligned
@@ -111,6 +111,25 @@ def test_dispatch_combine_empty_batch_is_a_no_op():
 ])
 def test_combine_rejects(args, status):
     assert ep.lib().ep_combine(*args) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((16, -1, 8, 16, 16, 16, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 0, 16, 16, 16, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 65, 16, 16, 16, 16, None, 0, None), ep.EP_ERR_UNSUPPORTED),
+    ((None, 4, 8, 16, 16, 16, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 8, None, 16, 16, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 8, 16, 16, 18, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),   # rank_row
+    ((16, 70000, 8, 16, 16, 16, 16, None, 0, None), ep.EP_ERR_INVALID_ARG),  # tiled, no ws
+])
+def test_rank_layout_rejects(args, status):
+    assert ep.lib().ep_get_rank_layout(*args) == status
+
+
+def test_rank_layout_workspace_sizes():
+    assert ep.ep_rank_layout_workspace_bytes(4096, 8) == 0
+    assert ep.ep_rank_layout_workspace_bytes(70000, 8) == ep.ep_layout_workspace_bytes(70000, 8, 8, 1)
+    assert ep.ep_rank_layout_workspace_bytes(70000, 8) > 0
 
 
 def test_read_error_rejects_null():
