@@ -204,9 +204,12 @@ __device__ __forceinline__ int rank_one(int e, int bits, int *hist_w) {
   return r;
 }
 
+// ids_smem (optional): the checked ids of the CTA's slots, indexed from
+// cta_beg, for the token-mask pass to read from shared memory.
 template <typename IdT>
 __device__ void rank_segment(const IdT *idx, long beg, long end, const Params &p,
-                             int32_t *d_err, int *hist_w, int32_t *slot_pos, SegRanks &sr) {
+                             int32_t *d_err, int *hist_w, int32_t *slot_pos, SegRanks &sr,
+                             short *ids_smem = nullptr, long cta_beg = 0) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, bits = p.id_bits;
   {
@@ -219,6 +222,8 @@ __device__ void rank_segment(const IdT *idx, long beg, long end, const Params &p
         const int e = check_id(v[b], E, d_err);
         const int r = rank_one(e, bits, hist_w);
         sr.packed[b] = e >= 0 ? (r << 10) | e : -1;
+        const long i = beg + 32 * b + lane;
+        if (ids_smem != nullptr && i < end) ids_smem[i - cta_beg] = static_cast<short>(e);
       }
     }
   }
@@ -231,22 +236,35 @@ __device__ void rank_segment(const IdT *idx, long beg, long end, const Params &p
       const long i = c0 + 32 * b + lane;
       const int e = check_id(v[b], E, d_err);
       const int r = rank_one(e, bits, hist_w);
-      if (i < end) slot_pos[i] = r;
+      if (i < end) {
+        slot_pos[i] = r;
+        if (ids_smem != nullptr) ids_smem[i - cta_beg] = static_cast<short>(e);
+      }
     }
   }
+}
+
+// The first row of expert e for this warp: base_w[e] (+ add1[e] + add2[e]
+// when given: the CTA's offset in the expert and the expert's offset).
+__device__ __forceinline__ int warp_base(int e, const int *base_w, const int *add1,
+                                         const int *add2) {
+  int b = base_w[e];
+  if (add1 != nullptr) b += add1[e] + add2[e];
+  return b;
 }
 
 template <typename IdT>
 __device__ void place_segment(const IdT *idx, long beg, long end, int k, int E,
                               const int *base_w, const SegRanks &sr, int32_t *slot_pos,
-                              int32_t *recv_src) {
+                              int32_t *recv_src, const int *add1 = nullptr,
+                              const int *add2 = nullptr) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int b = 0; b < kRegChunks; ++b) {
     const long i = beg + 32 * b + lane;
     if (i < end) {
       const int q = sr.packed[b];
-      const int pos = q >= 0 ? base_w[q & 1023] + (q >> 10) : -1;
+      const int pos = q >= 0 ? warp_base(q & 1023, base_w, add1, add2) + (q >> 10) : -1;
       slot_pos[i] = pos;
       if (pos >= 0) recv_src[pos] = static_cast<int32_t>(i / k);
     }
@@ -259,7 +277,7 @@ __device__ void place_segment(const IdT *idx, long beg, long end, int k, int E,
       const long i = c0 + 32 * b + lane;
       if (i < end) {
         const int e = check_id(v[b], E, nullptr);
-        const int pos = e >= 0 ? base_w[e] + slot_pos[i] : -1;
+        const int pos = e >= 0 ? warp_base(e, base_w, add1, add2) + slot_pos[i] : -1;
         slot_pos[i] = pos;
         if (pos >= 0) recv_src[pos] = static_cast<int32_t>(i / k);
       }
@@ -272,13 +290,20 @@ __device__ void place_segment(const IdT *idx, long beg, long end, int k, int E,
 // written by lane 0: the row is the warp's own).  Every thread of the
 // block runs the same number of rounds.
 template <typename IdT>
-__device__ void rank_mask(const Params &p, int t_beg, int t_end, int *hist_w) {
+__device__ void rank_mask(const Params &p, int t_beg, int t_end, int *hist_w,
+                          const short *ids_smem = nullptr) {
   const IdT *idx = static_cast<const IdT *>(p.idx);
   const int lane = threadIdx.x & 31;
   for (int t0 = t_beg; t0 < t_end; t0 += blockDim.x) {
     const int t = t0 + threadIdx.x;
     unsigned long long m = 0;
-    if (t < t_end) {
+    if (t < t_end && ids_smem != nullptr) {
+      const short *ids = ids_smem + static_cast<long>(t - t_beg) * p.k;
+      for (int j = 0; j < p.k; ++j) {
+        const int e = ids[j];
+        if (e >= 0) m |= 1ull << rank_of(e, p);
+      }
+    } else if (t < t_end) {
       const long base = static_cast<long>(t) * p.k;
       for (int j0 = 0; j0 < p.k; j0 += kIdBatch) {
         long long v[kIdBatch];
@@ -291,10 +316,10 @@ __device__ void rank_mask(const Params &p, int t_beg, int t_end, int *hist_w) {
           if (e >= 0) m |= 1ull << rank_of(e, p);
         }
       }
+    }
+    if (t < t_end && p.in_rank != nullptr) {
       uint8_t *row = p.in_rank + static_cast<long>(t) * p.R;
-      if (p.in_rank == nullptr) {
-        // mask layouts have no rank rows to write
-      } else if ((p.R & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 3) == 0) {
+      if ((p.R & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 3) == 0) {
         // 4 mask bytes per 32-bit store
         for (int r = 0; r < p.R; r += 4) {
           const unsigned b = static_cast<unsigned>(m >> r);
@@ -324,8 +349,34 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 
-int cluster_smem_bytes(int E, int R, int warps, int ctas) {
-  return (warps * (E + R + 1) + (ctas + 3) * (E + R)) * static_cast<int>(sizeof(int));
+// Slots per CTA up to which the CTA's checked ids are kept in shared
+// memory (int16) for the token-mask pass.
+constexpr long kStageIdsMax = 4096;
+
+int cluster_smem_bytes(int E, int R, int warps, int ctas, long staged_ids) {
+  return (warps * (E + R + 1) + (ctas + 2) * (E + R)) * static_cast<int>(sizeof(int)) +
+         static_cast<int>(((staged_ids * 2 + 15) / 16) * 16);
+}
+
+// Warp-wide exclusive scan of a[0..n) in place (32 elements per round) that
+// also writes the counts (cnt) and the exclusive offsets plus the total at
+// off[n] when those are given; returns the total.
+__device__ int scan_counts(int *a, int n, int32_t *cnt, int32_t *off) {
+  const int lane = threadIdx.x & 31;
+  int carry = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const int x = i < n ? a[i] : 0;
+    const int incl = warp_inclusive_scan(x);
+    if (i < n) {
+      a[i] = carry + incl - x;
+      if (cnt != nullptr) cnt[i] = x;
+      if (off != nullptr) off[i] = carry + incl - x;
+    }
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (off != nullptr && lane == 0) off[n] = carry;
+  return carry;
 }
 
 template <typename IdT>
@@ -338,12 +389,12 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
   extern __shared__ int smem[];
   const int E = p.E, R = p.R, C = E + R, ld = hist_ld(p);
   const int tid = threadIdx.x, nt = blockDim.x, w = tid >> 5, nw = nt >> 5;
-  int *hist = smem;               // [warps][E + R + 1]
-  int *all = hist + nw * ld;      // [ctas][C] every CTA's counts, pushed by each CTA
-  int *before = all + n_ctas * C; // [C] counts of the lower-ranked CTAs
-  int *tot = before + C;          // [C] totals, then exclusive offsets
-  int *base = tot + C;            // [C] first row of each expert for this CTA
-  __shared__ int s_kept;          // rows in use (all CTAs)
+  int *hist = smem;                // [warps][E + R + 1]
+  int *all = hist + nw * ld;       // [ctas][C] every CTA's counts, pushed by each CTA
+  int *before = all + n_ctas * C;  // [C] counts of the lower-ranked CTAs
+  int *tot = before + C;           // [C] totals, then exclusive offsets
+  short *ids_smem = reinterpret_cast<short *>(tot + C);  // staged ids (small CTAs)
+  __shared__ int s_kept;           // rows in use (all CTAs)
   const IdT *idx = static_cast<const IdT *>(p.idx);
 
   const int per_cta = (p.T + n_ctas - 1) / n_ctas;
@@ -351,6 +402,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
   const int t_end = min(p.T, t_beg + per_cta);
   const long s_beg = static_cast<long>(t_beg) * p.k;
   const long n = static_cast<long>(t_end - t_beg) * p.k;
+  const bool stage = static_cast<long>(per_cta) * p.k <= kStageIdsMax;
 
   for (int i = tid; i < nw * ld; i += nt) smem[i] = 0;
   __syncthreads();
@@ -359,12 +411,14 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
   const long seg_beg = warp_slice(n, w, nw, &seg_end);
   SegRanks sr;
   rank_segment(idx, s_beg + seg_beg, s_beg + seg_end, p, p.d_err, hist + w * ld, p.slot_pos,
-               sr);
-  rank_mask<IdT>(p, t_beg, t_end, hist + w * ld);
+               sr, stage ? ids_smem : nullptr, s_beg);
+  if (stage) __syncthreads();  // every warp's ids are in shared memory
+  rank_mask<IdT>(p, t_beg, t_end, hist + w * ld, stage ? ids_smem : nullptr);
   __syncthreads();
   if (n_ctas > 1) cluster_wait();  // every CTA of the cluster is running
-  // one thread per column: exclusive prefix over this CTA's warps, and the
-  // CTA's count pushed into row `rank` of every CTA's `all`
+  // one thread per column: exclusive prefix over this CTA's warps; the
+  // CTA's count goes to row `rank` of every CTA's `all` (or straight to
+  // `tot` when the CTA is alone)
   for (int c = tid; c < C; c += nt) {
     int run = 0;
     for (int v = 0; v < nw; ++v) {
@@ -375,53 +429,38 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
     if (n_ctas > 1) {
       for (int q = 0; q < n_ctas; ++q) cluster.map_shared_rank(all, q)[rank * C + c] = run;
     } else {
-      all[c] = run;
+      before[c] = 0;
+      tot[c] = run;
     }
   }
-  if (n_ctas > 1)
+  if (n_ctas > 1) {
     cluster.sync();  // all pushes done and visible; nothing remote after this
-  else
-    __syncthreads();
-  for (int c = tid; c < C; c += nt) {
-    int b = 0, a = 0;
-    for (int r = 0; r < n_ctas; ++r) {
-      const int v = all[r * C + c];
-      b += r < rank ? v : 0;
-      a += v;
-    }
-    before[c] = b;
-    tot[c] = a;
-  }
-  __syncthreads();
-  if (rank == 0)
     for (int c = tid; c < C; c += nt) {
-      if (c < E) p.cnt_e[c] = tot[c];
-      else if (p.cnt_r != nullptr) p.cnt_r[c - E] = tot[c];
+      int b = 0, a = 0;
+      for (int r = 0; r < n_ctas; ++r) {
+        const int v = all[r * C + c];
+        b += r < rank ? v : 0;
+        a += v;
+      }
+      before[c] = b;
+      tot[c] = a;
     }
-  // warp 0 scans the expert totals, warp 1 the rank totals
+  }
+  __syncthreads();
+  // warp 0 scans the expert totals, warp 1 the rank totals; CTA 0 writes
+  // the counts and offsets as it goes
   if (w == 0) {
-    const int n_kept = warp_exclusive_scan_smem(tot, E);
-    if (tid == 0) {
-      s_kept = n_kept;
-      if (rank == 0) p.off_e[E] = n_kept;
-    }
+    const int n_kept =
+        scan_counts(tot, E, rank == 0 ? p.cnt_e : nullptr, rank == 0 ? p.off_e : nullptr);
+    if (tid == 0) s_kept = n_kept;
   } else if (w == 1) {
-    const int n_tok = warp_exclusive_scan_smem(tot + E, R);
-    if (rank == 0 && (tid & 31) == 0 && p.off_r != nullptr) p.off_r[R] = n_tok;
+    scan_counts(tot + E, R, rank == 0 ? p.cnt_r : nullptr, rank == 0 ? p.off_r : nullptr);
   }
   __syncthreads();
-  for (int c = tid; c < C; c += nt) {
-    if (rank == 0) {
-      if (c < E) p.off_e[c] = tot[c];
-      else if (p.off_r != nullptr) p.off_r[c - E] = tot[c];
-    }
-    if (c < E) base[c] = tot[c] + before[c];
-  }
-  __syncthreads();
-  add_column_bases(hist, ld, E, nw, base);
-  __syncthreads();
+  // row = this warp's count of earlier slots + the CTA's offset in the
+  // expert (before) + the expert's offset (tot)
   place_segment(idx, s_beg + seg_beg, s_beg + seg_end, p.k, E, hist + w * ld, sr, p.slot_pos,
-                p.recv_src);
+                p.recv_src, before, tot);
   // rows nobody fills (past the kept ones)
   const long N = static_cast<long>(p.T) * p.k;
   for (long r = s_kept + static_cast<long>(rank) * nt + tid; r < N;
@@ -635,15 +674,18 @@ cudaError_t launch_cluster(Params p, cudaStream_t s, int *launches) {
   const int threads = N <= kSmallSlots ? kSmallThreads : kClusterThreads;
   cudaError_t err = raise_dynamic_smem(
       reinterpret_cast<const void *>(kern),
-      cluster_smem_bytes(p.E, p.R, kClusterWarps, kMaxClusterCtas));
+      cluster_smem_bytes(p.E, p.R, kClusterWarps, kMaxClusterCtas, kStageIdsMax));
   if (err != cudaSuccess) return err;
   long want = (N + kSlotsPerClusterCta - 1) / kSlotsPerClusterCta;
   if (want < 1) want = 1;
   const int cap = want > 8 ? max_cluster_ctas<IdT>(cluster_smem_bytes(
-                                 p.E, p.R, threads / kWarp, kMaxClusterCtas))
+                                 p.E, p.R, threads / kWarp, kMaxClusterCtas, kStageIdsMax))
                            : 8;
   const int n_ctas = static_cast<int>(want < cap ? want : cap);
-  const int smem = cluster_smem_bytes(p.E, p.R, threads / kWarp, n_ctas);
+  // slots of the largest CTA: staged in shared memory when small enough
+  const long per_cta_slots = static_cast<long>((p.T + n_ctas - 1) / n_ctas) * p.k;
+  const int smem = cluster_smem_bytes(p.E, p.R, threads / kWarp, n_ctas,
+                                      per_cta_slots <= kStageIdsMax ? per_cta_slots : 0);
   ++*launches;
   return launch_pdl(kern, dim3(n_ctas), dim3(threads), smem, s, n_ctas, p);
 }
