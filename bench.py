@@ -363,7 +363,7 @@ def bench_ours(args, world, rank, device):
 KERNEL_SOURCES = {
     "layout": ("layout.cu", "ep_internal.cuh"),
     "dispatch_bf16": ("dispatch.cu", "ep_internal.cuh"),
-    "dispatch_fp8": ("dispatch.cu", "ep_internal.cuh"),
+    "dispatch_fp8": ("dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
     "combine": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),
 }
 
@@ -465,28 +465,66 @@ def bench_decode(ep, device, world, iters=200):
     stream.synchronize()
     us_stream = a.elapsed_time(b) * 1e3 / iters
 
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        st.run(stream, fp8_only=True)
-    with torch.cuda.stream(stream):
-        for _ in range(20):
-            g.replay()
-        a.record(stream)
-        for _ in range(iters):
-            g.replay()
-        b.record(stream)
-    stream.synchronize()
-    us_graph = a.elapsed_time(b) * 1e3 / iters
-    del g
+    def graph_us(fn):
+        """Device time of one replay of a CUDA graph holding fn's launches."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        with torch.cuda.stream(stream):
+            for _ in range(20):
+                g.replay()
+            a.record(stream)
+            for _ in range(iters):
+                g.replay()
+            b.record(stream)
+        stream.synchronize()
+        del g
+        return a.elapsed_time(b) * 1e3 / iters
+
+    c = cfg
+
+    def layout_dispatch():
+        ep.ep_layout_dispatch(st.idx, c.E, c.R, st.x, True, out=st.layout, recv=st.recv_q,
+                              recv_scale=st.recv_s, ws=st.ws, d_err=st.d_err, stream=stream)
+
+    def combine():
+        ep.ep_combine(st.recv, st.layout.slot_pos, st.w, out=st.out, d_err=st.d_err,
+                      stream=stream)
+
+    def fused_call():
+        layout_dispatch()
+        combine()
+
+    us_graph = graph_us(lambda: st.run(stream, fp8_only=True))
+    us_fused = graph_us(fused_call)
+    # each kernel of the call alone, replayed from its own graph
+    parts = {
+        "layout": lambda: ep.ep_get_layout(st.idx, c.E, c.R, out=st.layout, ws=st.ws,
+                                           d_err=st.d_err, stream=stream),
+        "dispatch_fp8": lambda: ep.ep_dispatch(st.x, st.layout.slot_pos, fp8=True,
+                                               recv=st.recv_q, recv_scale=st.recv_s,
+                                               d_err=st.d_err, stream=stream),
+        "layout_dispatch_fp8": layout_dispatch,
+        "combine": combine,
+    }
+    part_us = {name: round(max_over_ranks(graph_us(fn), world, device), 2)
+               for name, fn in parts.items()}
+    if ep.ep_read_error(st.d_err, stream) != 0:
+        raise RuntimeError("the device reported an error in the decode calls")
     us_stream = max_over_ranks(us_stream, world, device)
     us_graph = max_over_ranks(us_graph, world, device)
+    us_fused = max_over_ranks(us_fused, world, device)
     nb = decode_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R)
     return {"workload": "decode: T=128, H=7168, E=256/R=8, top-8, FP8 dispatch; "
                         "call = layout + FP8 dispatch + combine",
             "us_per_call_graph": round(us_graph, 2),
+            "us_per_call_graph_fused": round(us_fused, 2),
+            "fused": "ep_layout_dispatch (layout + FP8 dispatch, one kernel) + combine",
+            "us_per_kernel_graph": part_us,
             "us_per_call_stream": round(us_stream, 2),
             "bytes_per_call": nb,
             "GB/s_graph": round(nb / (us_graph * 1e-6) / 1e9, 1),
+            "GB/s_graph_fused": round(nb / (us_fused * 1e-6) / 1e9, 1),
             "l2": "warm (back-to-back calls; the working set fits in L2)",
             "pages_context_us": 163.0}
 

@@ -10,6 +10,7 @@ CPU path: if the library is missing, calls raise ``EPLibraryError``.
     recv = ep_dispatch(x, layout.slot_pos)            # bf16 rows
     q, scale = ep_dispatch(x, layout.slot_pos, fp8=True)
     out = ep_combine(y, layout.slot_pos, w)           # gate-weighted sum
+    layout, (q, scale) = ep_layout_dispatch(idx, E, R, x, fp8=True)  # one launch
 """
 from __future__ import annotations
 
@@ -22,7 +23,7 @@ import torch
 __all__ = ["EPError", "EPLibraryError", "Layout", "RankLayout", "ep_get_layout",
            "ep_get_rank_layout", "ep_rank_layout_workspace_bytes",
            "ep_get_layout_noalloc", "EP_NOALLOC_SCRATCH_BYTES",
-           "ep_dispatch", "ep_combine", "ep_read_error",
+           "ep_dispatch", "ep_combine", "ep_read_error", "ep_layout_dispatch",
            "ep_layout_workspace_bytes", "ep_kernel_launches", "lib",
            "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_UNSUPPORTED", "EP_ERR_CUDA",
            "EP_ERR_INDEX", "EP_ERR_TIMEOUT", "LIB_PATH"]
@@ -68,6 +69,8 @@ _SIGNATURES = {
                                _vp, _vp, _vp, _vp], _i),
     "ep_rank_layout_workspace_bytes": ([_i, _i], _sz),
     "ep_get_rank_layout": ([_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i),
+    "ep_layout_dispatch": ([_vp, _i, _i, _i, _i, _i, _vp, _i, _i, _vp, _vp, _vp, _vp,
+                            _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _vp, _vp], _i),
 }
 
 
@@ -248,6 +251,43 @@ def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
                              _ptr(recv), _ptr(recv_scale) if fp8 else None,
                              num_sms, _ptr(d_err), _stream(stream)))
     return (recv, recv_scale) if fp8 else recv
+
+
+def ep_layout_dispatch(idx: torch.Tensor, E: int, R: int, x: torch.Tensor,
+                       fp8: bool = False, *, out: Optional[Layout] = None,
+                       recv: Optional[torch.Tensor] = None,
+                       recv_scale: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None, num_sms: int = 0,
+                       d_err: Optional[torch.Tensor] = None, stream=None):
+    """ep_get_layout then ep_dispatch, in one kernel launch for small
+    batches (a decode step).  Returns ``(layout, recv)`` or, with ``fp8``,
+    ``(layout, (recv_q, recv_scale))``, bit-identical to the two calls."""
+    _need_cuda("idx", idx)
+    _need_cuda("x", x)
+    if idx.dtype not in (torch.int64, torch.int32) or idx.dim() != 2:
+        raise ValueError("idx must be a 2-D int64 or int32 tensor")
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[0] != idx.shape[0]:
+        raise ValueError("x must be a bf16 [T, H] tensor with idx's T")
+    T, k = idx.shape
+    H = x.shape[1]
+    if out is None:
+        out = empty_layout(T, k, E, R, idx.device)
+    if recv is None:
+        recv = torch.empty((T * k, H), device=x.device,
+                           dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16)
+    if fp8 and recv_scale is None:
+        recv_scale = torch.empty((T * k, H // 128), device=x.device, dtype=torch.float32)
+    need = ep_layout_workspace_bytes(T, k, E, R)
+    if ws is None and need > 0:
+        ws = torch.zeros(need, dtype=torch.uint8, device=idx.device)
+    _check(lib().ep_layout_dispatch(
+        _ptr(idx), int(idx.dtype == torch.int64), T, k, E, R, _ptr(x), H, int(bool(fp8)),
+        _ptr(out.cnt_e), _ptr(out.cnt_r), _ptr(out.in_rank), _ptr(out.off_e),
+        _ptr(out.off_r), _ptr(out.slot_pos), _ptr(out.recv_src), _ptr(recv),
+        _ptr(recv_scale) if fp8 else None, _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), num_sms, _ptr(d_err),
+        _stream(stream)))
+    return out, ((recv, recv_scale) if fp8 else recv)
 
 
 def ep_combine(y: torch.Tensor, slot_pos: torch.Tensor, w: Optional[torch.Tensor], *,

@@ -130,7 +130,7 @@ cudaError_t raise_dynamic_smem(const void *kernel, int bytes) {
 
 extern "C" {
 
-int ep_abi_version(void) { return 2; }
+int ep_abi_version(void) { return 3; }
 
 const char *ep_last_error_string(void) { return g_err; }
 
@@ -150,6 +150,30 @@ static ep_status_t check_layout_sizes(const char *fn, int T, int k, int E, int R
   if (static_cast<long long>(T) * k > 0x7fffffffLL)
     return fail(EP_ERR_UNSUPPORTED, "%s: T*k does not fit int32", fn);
   return EP_OK;
+}
+
+static ep::LayoutArgs expert_layout_args(const void *idx, int idx_is_int64, int T, int k, int E,
+                                        int R, int32_t *cnt_e, int32_t *cnt_r,
+                                        uint8_t *in_rank, int32_t *off_e, int32_t *off_r,
+                                        int32_t *slot_pos, int32_t *recv_src, void *ws,
+                                        int32_t *d_err) {
+  ep::LayoutArgs a{};
+  a.idx = idx;
+  a.id_kind = idx_is_int64 ? ep::kIdsInt64 : ep::kIdsInt32;
+  a.T = T;
+  a.k = k;
+  a.E = E;
+  a.R = R;
+  a.cnt_e = cnt_e;
+  a.cnt_r = cnt_r;
+  a.off_e = off_e;
+  a.off_r = off_r;
+  a.slot_pos = slot_pos;
+  a.recv_src = recv_src;
+  a.in_rank = in_rank;
+  a.ws = ws;
+  a.d_err = d_err;
+  return a;
 }
 
 size_t ep_layout_workspace_bytes(int T, int k, int E, int R) {
@@ -184,22 +208,9 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
     if (ws_bytes < need)
       return fail(EP_ERR_INVALID_ARG, "%s: ws_bytes=%zu < %zu needed", fn, ws_bytes, need);
   }
-  ep::LayoutArgs a{};
-  a.idx = idx;
-  a.id_kind = idx_is_int64 ? ep::kIdsInt64 : ep::kIdsInt32;
-  a.T = T;
-  a.k = k;
-  a.E = E;
-  a.R = R;
-  a.cnt_e = cnt_e;
-  a.cnt_r = cnt_r;
-  a.off_e = off_e;
-  a.off_r = off_r;
-  a.slot_pos = slot_pos;
-  a.recv_src = recv_src;
-  a.in_rank = in_rank;
-  a.ws = ws;
-  a.d_err = d_err;
+  const ep::LayoutArgs a = expert_layout_args(idx, idx_is_int64, T, k, E, R, cnt_e, cnt_r,
+                                               in_rank, off_e, off_r, slot_pos, recv_src, ws,
+                                               d_err);
   int n = 0;
   const cudaError_t e = ep::launch_layout(a, static_cast<cudaStream_t>(stream), &n);
   g_launches += n;
@@ -275,6 +286,50 @@ ep_status_t ep_dispatch(const void *x, int T, int H, int k,
   const cudaError_t e =
       fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale, num_sms, d_err, s, &n)
           : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, num_sms, d_err, s, &n);
+  g_launches += n;
+  return from_cuda(e, fn);
+}
+
+ep_status_t ep_layout_dispatch(const void *idx, int idx_is_int64, int T, int k, int E, int R,
+                               const void *x, int H, int fp8, int32_t *cnt_e, int32_t *cnt_r,
+                               uint8_t *in_rank, int32_t *off_e, int32_t *off_r,
+                               int32_t *slot_pos, int32_t *recv_src, void *recv,
+                               float *recv_scale, void *ws, size_t ws_bytes, int num_sms,
+                               int32_t *d_err, void *stream) {
+  static const char fn[] = "ep_layout_dispatch";
+  ep_status_t st = ep::check_layout_args(fn, idx, idx_is_int64, T, k, E, R, cnt_e, cnt_r,
+                                         in_rank, off_e, off_r, slot_pos, recv_src, d_err);
+  if (st != EP_OK) return st;
+  st = check_rows(fn, T, H, k, num_sms);
+  if (st != EP_OK) return st;
+  if (fp8 && H % 128 != 0)
+    return fail(EP_ERR_UNSUPPORTED, "%s: fp8 needs H %% 128 == 0 (H=%d)", fn, H);
+  if (T > 0) {
+    EP_REQUIRE_PTR(fn, x, 16);
+    EP_REQUIRE_PTR(fn, recv, 16);
+    if (fp8) EP_REQUIRE_PTR(fn, recv_scale, 4);
+  }
+  const size_t need = ep::layout_workspace_bytes(T, k, E, R);
+  if (need > 0) {
+    EP_REQUIRE_PTR(fn, ws, 16);
+    if (ws_bytes < need)
+      return fail(EP_ERR_INVALID_ARG, "%s: ws_bytes=%zu < %zu needed", fn, ws_bytes, need);
+  }
+  const ep::LayoutArgs a = expert_layout_args(idx, idx_is_int64, T, k, E, R, cnt_e, cnt_r,
+                                               in_rank, off_e, off_r, slot_pos, recv_src, ws,
+                                               d_err);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int n = 0;
+  cudaError_t e;
+  if (ep::layout_dispatch_fusable(T, k, E, R, H, fp8 != 0, recv_scale)) {
+    e = ep::launch_layout_dispatch(a, x, H, fp8 != 0, recv, recv_scale, num_sms, s, &n);
+  } else {
+    e = ep::launch_layout(a, s, &n);
+    if (e == cudaSuccess)
+      e = fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale, num_sms, d_err,
+                                        s, &n)
+              : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, num_sms, d_err, s, &n);
+  }
   g_launches += n;
   return from_cuda(e, fn);
 }

@@ -93,6 +93,14 @@ cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
                                 float *recv_scale, int num_sms, int32_t *d_err,
                                 cudaStream_t s, int *launches);
+// Layout and dispatch in one launch (small batches; see layout_dispatch.cu).
+// layout_dispatch_fusable says whether the sizes (and, for FP8, the scale
+// pointer's alignment) fit that kernel.
+bool layout_dispatch_fusable(int T, int k, int E, int R, int H, bool fp8,
+                             const float *recv_scale);
+cudaError_t launch_layout_dispatch(const LayoutArgs &la, const void *x, int H, bool fp8,
+                                   void *recv, float *recv_scale, int num_sms, cudaStream_t s,
+                                   int *launches);
 cudaError_t launch_combine(const void *y, int T, int H, int k,
                            const int32_t *slot_pos, const float *w, void *out,
                            int num_sms, int32_t *d_err, cudaStream_t s,

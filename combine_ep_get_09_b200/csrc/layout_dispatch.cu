@@ -1,0 +1,379 @@
+// layout_dispatch.cu -- the dispatch layout and the dispatch of the same
+// batch in ONE launch, for small batches such as a decode step.
+//
+// DeepEP keeps separate low-latency kernels for small decode batches
+// (dataforcee.us rewrite, "Technological Views and Benefits": 128 tokens,
+// eight experts).  Inside one GPU such a step is bound by launch and
+// dependency latency, not by bytes, so this path drops the layout launch
+// and the wait between it and the dispatch: every CTA computes the whole
+// layout of the batch in its own shared memory from the ids (a few KB,
+// served by L2 after the first CTA reads them), with no CTA ever waiting on
+// another, then dispatches its own contiguous range of tokens and writes
+// the layout entries of those tokens; CTA 0 also writes the counts and
+// offsets.  The token rows are bulk-loaded (cp.async.bulk) before the
+// layout work starts, so the layout hides under the row loads.
+//
+// The layout in shared memory is one token bit set per expert: bit t % 32
+// of mask[e][t / 32] is set when token t chose expert e.  The receive row
+// of slot (t, j) with expert e is off_e[e] + (tokens before t that chose e),
+// a popcount of the set below bit t -- the stable token-major order of the
+// unfused layout.  A token naming one expert twice (two slots, as the
+// unfused path accepts) is seen while the sets are built; the ranks are
+// then counted over the flat slot order instead.  Results are bit-identical
+// to ep_get_layout followed by ep_dispatch.
+#include <cuda_bf16.h>
+
+#include "bulk.cuh"
+#include "ep_internal.cuh"
+#include "fp8.cuh"
+
+namespace ep {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / kWarp;
+constexpr int kStages = 2;             // token rows in flight per CTA
+constexpr long kMaxSlots = 8192;       // T * k of the fused path
+constexpr long kMaxMaskBytes = 32768;  // E * ceil(T / 32) * 4
+constexpr int kMaxH = 16384;
+
+__host__ __device__ constexpr int align16(long b) { return static_cast<int>((b + 15) & ~15L); }
+
+// Byte offsets of the dynamic shared memory regions (host and device agree).
+struct SmemMap {
+  int in, out_q, out_s, mask, cnt, off, cnt_r, ids, total;
+};
+
+__host__ __device__ inline SmemMap smem_map(int T, int k, int E, int R, int H, bool fp8) {
+  SmemMap m;
+  const long W = (T + 31) / 32;
+  int o = 0;
+  m.in = o;     o += kStages * 2 * H;           // bf16 rows: 2H is a multiple of 16
+  m.out_q = o;  o += fp8 ? H : 0;               // e4m3 row
+  m.out_s = o;  o += fp8 ? H / 32 : 0;          // H / 128 fp32 scales
+  m.mask = o;   o += align16(E * W * 4);
+  m.cnt = o;    o += align16(static_cast<long>(E) * 4);
+  m.off = o;    o += align16(static_cast<long>(E + 1) * 4);
+  m.cnt_r = o;  o += align16(static_cast<long>(R) * 4);
+  m.ids = o;    o += align16(static_cast<long>(T) * k * 2);
+  m.total = o;
+  return m;
+}
+
+struct FusedArgs {
+  const void *idx;
+  int T, k, E, R, G, H, W;
+  const uint4 *x;
+  int32_t *cnt_e, *cnt_r, *off_e, *off_r, *slot_pos, *recv_src;
+  uint8_t *in_rank;
+  unsigned char *recv;  // bf16 [T*k, H] or e4m3 [T*k, H]
+  float *recv_scale;    // [T*k, H / 128] (FP8)
+  int32_t *d_err;
+  int per_cta;          // tokens per CTA
+};
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// out[0..n) = exclusive scan of in[0..n), out[n] = total, by the whole CTA
+// (each thread a contiguous run of ceil(n / kThreads) entries).
+__device__ void block_exclusive_scan(const int *in, int *out, int n, int *warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n + kThreads - 1) / kThreads;
+  const int b = min(n, tid * per), e = min(n, b + per);
+  int local = 0;
+  for (int q = b; q < e; ++q) local += in[q];
+  const int incl = warp_incl_scan(local);
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < kWarps ? warp_tot[lane] : 0;
+    const int iv = warp_incl_scan(v);
+    if (lane < kWarps) warp_tot[lane] = iv - v;
+    if (lane == kWarps - 1) out[n] = iv;
+  }
+  __syncthreads();
+  int run = warp_tot[warp] + incl - local;
+  for (int q = b; q < e; ++q) {
+    out[q] = run;
+    run += in[q];
+  }
+}
+
+template <typename IdT, bool kFp8>
+__global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(const FusedArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const SmemMap sm = smem_map(a.T, a.k, a.E, a.R, a.H, kFp8);
+  unsigned char *in_buf = smem + sm.in;
+  unsigned char *out_q = smem + sm.out_q;
+  float *out_s = reinterpret_cast<float *>(smem + sm.out_s);
+  unsigned *mask = reinterpret_cast<unsigned *>(smem + sm.mask);
+  int *cnt = reinterpret_cast<int *>(smem + sm.cnt);
+  int *off = reinterpret_cast<int *>(smem + sm.off);
+  int *cnt_r = reinterpret_cast<int *>(smem + sm.cnt_r);
+  int16_t *ids = reinterpret_cast<int16_t *>(smem + sm.ids);
+  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ int rows[2][EP_MAX_K];
+  __shared__ int warp_tot[kWarps];
+  __shared__ int dup;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = a.T, k = a.k, E = a.E, R = a.R, G = a.G, H = a.H, W = a.W;
+  const long N = static_cast<long>(T) * k;
+  const int first = blockIdx.x * a.per_cta;
+  const int n_mine = max(0, min(T, first + a.per_cta) - first);
+  const int in_bytes = 2 * H;
+  const bool lead = blockIdx.x == 0;
+
+  pdl_trigger();
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    mbar_init_fence();
+    dup = 0;
+  }
+  for (int q = tid; q < E * W; q += kThreads) mask[q] = 0u;
+  for (int q = tid; q < E; q += kThreads) cnt[q] = 0;
+  for (int q = tid; q < R; q += kThreads) cnt_r[q] = 0;
+  __syncthreads();
+  pdl_wait();  // ids and rows come from the previous kernel on the stream
+
+  // thread 0: token first + i -> input stage i % kStages
+  auto issue = [&](int i) {
+    const int s = i % kStages;
+    mbar_arrive_expect_tx(&full[s], in_bytes);
+    bulk_load(in_buf + s * in_bytes, a.x + static_cast<long>(first + i) * (H >> 3), in_bytes,
+              &full[s]);
+  };
+  if (tid == 0)
+    for (int i = 0; i < min(kStages, n_mine); ++i) issue(i);
+
+  // 1. ids -> per-expert token sets and slot counts (bad ids reported once)
+  const IdT *idx = static_cast<const IdT *>(a.idx);
+  constexpr int kBatch = 4;
+  for (long base = 0; base < N; base += kBatch * kThreads) {
+    long long v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const long i = base + u * kThreads + tid;
+      v[u] = i < N ? static_cast<long long>(idx[i]) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const long i = base + u * kThreads + tid;
+      if (i >= N) continue;
+      int e = -1;
+      if (v[u] >= 0 && v[u] < E)
+        e = static_cast<int>(v[u]);
+      else if (v[u] != -1 && lead && a.d_err != nullptr)
+        atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_INDEX);
+      ids[i] = static_cast<int16_t>(e);
+      if (e >= 0) {
+        const int t = static_cast<int>(i / k);
+        const unsigned bit = 1u << (t & 31);
+        if (atomicOr(&mask[e * W + (t >> 5)], bit) & bit) dup = 1;
+        atomicAdd(&cnt[e], 1);
+      }
+    }
+  }
+  __syncthreads();
+
+  // 2. offsets; CTA 0 also counts the tokens of each rank
+  block_exclusive_scan(cnt, off, E, warp_tot);
+  if (lead) {
+    for (int q = tid; q < R * W; q += kThreads) {
+      const int r = q / W, w = q - r * W;
+      unsigned m = 0u;
+      for (int g = 0; g < G; ++g) m |= mask[(r * G + g) * W + w];
+      if (m != 0u) atomicAdd(&cnt_r[r], __popc(m));
+    }
+  }
+  __syncthreads();
+  const int n_eff = off[E];
+  if (lead) {
+    for (int q = tid; q < E; q += kThreads) {
+      a.cnt_e[q] = cnt[q];
+      a.off_e[q] = off[q];
+    }
+    if (tid == 0) a.off_e[E] = n_eff;
+    if (warp == kWarps - 1) {  // R <= 64
+      int carry = 0;
+      for (int b = 0; b < R; b += 32) {
+        const int r = b + lane;
+        const int c = r < R ? cnt_r[r] : 0;
+        const int incl = warp_incl_scan(c);
+        if (r < R) {
+          a.cnt_r[r] = c;
+          a.off_r[r] = carry + incl - c;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) a.off_r[R] = carry;
+    }
+  }
+  // receive rows no slot points at
+  for (long r = n_eff + static_cast<long>(blockIdx.x) * kThreads + tid; r < N;
+       r += static_cast<long>(gridDim.x) * kThreads)
+    a.recv_src[r] = -1;
+
+  // 3. this CTA's tokens: rows and layout entries, then the dispatch
+  int i = 0;
+  bool timed_out = false;
+  for (; i < n_mine; ++i) {
+    const int t = first + i;
+    const int s = i % kStages;
+    const int rb = i & 1;
+    for (int j = warp; j < k; j += kWarps) {  // a warp per slot
+      const int e = ids[t * k + j];
+      int before = 0;
+      if (e >= 0) {
+        int c = 0;
+        if (!dup) {  // tokens before t that chose e
+          const unsigned *me = mask + e * W;
+          const int wt = t >> 5;
+          for (int w = lane; w < wt; w += 32) c += __popc(me[w]);
+          if (lane == 0) c += __popc(me[wt] & ((1u << (t & 31)) - 1u));
+        } else {  // slots before (t, j) in token-major order with expert e
+          const int flat = t * k + j;
+          for (int q = lane; q < flat; q += 32) c += ids[q] == e;
+        }
+        before = warp_sum(c);
+      }
+      if (lane == 0) {
+        const int row = e >= 0 ? off[e] + before : -1;
+        rows[rb][j] = row;
+        a.slot_pos[static_cast<long>(t) * k + j] = row;
+        if (row >= 0) a.recv_src[row] = t;
+      }
+    }
+    for (int r = tid; r < R; r += kThreads) {
+      int in = 0;
+      for (int j = 0; j < k; ++j) {
+        const int e = ids[t * k + j];
+        in |= e >= 0 && e / G == r;
+      }
+      a.in_rank[static_cast<long>(t) * R + r] = static_cast<uint8_t>(in);
+    }
+    if (kFp8 && tid == 0) bulk_wait_read<0>();  // the previous token's stores left out_q
+    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1));
+    if (__syncthreads_or(!ok)) {
+      timed_out = true;
+      break;
+    }
+    if (kFp8) {
+      const uint4 *xin = reinterpret_cast<const uint4 *>(in_buf + s * in_bytes);
+      uint2 *qo = reinterpret_cast<uint2 *>(out_q);
+      // a half-warp per 128-channel block; whole warps share the loop bound
+      // because H / 8 is a multiple of 64
+      for (int v = tid; v < (H >> 3); v += kThreads) {
+        float sc;
+        qo[v] = quantize_block_lane(xin[v], &sc);
+        if ((tid & 15) == 0) out_s[v >> 4] = sc;
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        const int nb = H >> 7;
+        for (int j = 0; j < k; ++j) {
+          const int row = rows[rb][j];
+          if (row < 0) continue;
+          bulk_store(a.recv + static_cast<long>(row) * H, out_q, H);
+          bulk_store(a.recv_scale + static_cast<long>(row) * nb, out_s, 4 * nb);
+        }
+        bulk_commit();
+        if (i + kStages < n_mine) issue(i + kStages);  // stage s was read by the cast only
+      }
+    } else if (tid == 0) {
+      for (int j = 0; j < k; ++j) {
+        const int row = rows[rb][j];
+        if (row < 0) continue;
+        bulk_store(a.recv + static_cast<long>(row) * in_bytes, in_buf + s * in_bytes, in_bytes);
+      }
+      bulk_commit();
+      if (i + kStages < n_mine) {
+        bulk_wait_read<0>();  // the stores above have read stage s
+        issue(i + kStages);
+      }
+    }
+  }
+  if (tid == 0) {
+    if (timed_out) {
+      if (a.d_err != nullptr) atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_TIMEOUT);
+      // let the row loads still in flight land before the CTA's memory goes away
+      for (int q = i; q < min(n_mine, i + kStages); ++q)
+        mbar_wait_bounded(&full[q % kStages], static_cast<unsigned>((q / kStages) & 1));
+    }
+    bulk_wait<0>();
+  }
+}
+
+template <typename IdT, bool kFp8>
+cudaError_t launch_fused(const FusedArgs &base, int num_sms, cudaStream_t s) {
+  auto kern = layout_dispatch_kernel<IdT, kFp8>;
+  const int smem = smem_map(base.T, base.k, base.E, base.R, base.H, kFp8).total;
+  cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
+  if (err != cudaSuccess) return err;
+  // a CTA per token, capped at the CTAs that fit at once; no CTA left empty
+  const long cap = persistent_grid(reinterpret_cast<const void *>(kern), kThreads, smem,
+                                   static_cast<long>(base.T) * kWarps, num_sms);
+  FusedArgs a = base;
+  a.per_cta = static_cast<int>((base.T + cap - 1) / cap);
+  const int grid = (base.T + a.per_cta - 1) / a.per_cta;
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, 1, a);
+}
+
+}  // namespace
+
+bool layout_dispatch_fusable(int T, int k, int E, int R, int H, bool fp8,
+                             const float *recv_scale) {
+  (void)R;
+  if (T < 1 || static_cast<long>(T) * k > kMaxSlots || H > kMaxH) return false;
+  if (static_cast<long>(E) * ((T + 31) / 32) * 4 > kMaxMaskBytes) return false;
+  if (fp8 && (H % 512 != 0 || reinterpret_cast<uintptr_t>(recv_scale) % 16 != 0)) return false;
+  return true;
+}
+
+cudaError_t launch_layout_dispatch(const LayoutArgs &la, const void *x, int H, bool fp8,
+                                   void *recv, float *recv_scale, int num_sms, cudaStream_t s,
+                                   int *launches) {
+  FusedArgs a{};
+  a.idx = la.idx;
+  a.T = la.T;
+  a.k = la.k;
+  a.E = la.E;
+  a.R = la.R;
+  a.G = la.E / la.R;
+  a.H = H;
+  a.W = (la.T + 31) / 32;
+  a.x = static_cast<const uint4 *>(x);
+  a.cnt_e = la.cnt_e;
+  a.cnt_r = la.cnt_r;
+  a.off_e = la.off_e;
+  a.off_r = la.off_r;
+  a.slot_pos = la.slot_pos;
+  a.recv_src = la.recv_src;
+  a.in_rank = la.in_rank;
+  a.recv = static_cast<unsigned char *>(recv);
+  a.recv_scale = recv_scale;
+  a.d_err = la.d_err;
+  ++*launches;
+  if (la.id_kind == kIdsInt64)
+    return fp8 ? launch_fused<long long, true>(a, num_sms, s)
+               : launch_fused<long long, false>(a, num_sms, s);
+  return fp8 ? launch_fused<int32_t, true>(a, num_sms, s)
+             : launch_fused<int32_t, false>(a, num_sms, s);
+}
+
+}  // namespace ep

@@ -147,6 +147,36 @@ ep_status_t ep_dispatch(const void *x, int T, int H, int k,
                         void *stream);
 
 /*
+ * ep_layout_dispatch -- ep_get_layout followed by ep_dispatch, with the
+ * same arguments and bit-identical outputs, in one kernel launch when the
+ * batch is small.
+ *
+ * DeepEP serves small decode batches with separate low-latency kernels
+ * (dataforcee.us rewrite, "Technological Views and Benefits": 128 tokens,
+ * eight experts); on one GPU their cost is launch and dependency latency.
+ * When T*k <= 8192, E * ceil(T/32) * 4 <= 32 KiB and H <= 16384 (for FP8
+ * also H % 512 == 0 and a 16-byte aligned recv_scale), one kernel computes
+ * the layout redundantly in every CTA's shared memory, writes it, and
+ * dispatches; otherwise the call enqueues the two kernels of ep_get_layout
+ * and ep_dispatch (ep_kernel_launches tells which ran).
+ *
+ * idx .. recv_src, ws, ws_bytes: as ep_get_layout (ws is needed only when
+ * ep_layout_workspace_bytes(T, k, E, R) > 0, i.e. for T*k > 2^19).
+ * x, H, fp8, recv, recv_scale, num_sms: as ep_dispatch.
+ * d_err receives EP_ERR_INDEX for a bad id and EP_ERR_TIMEOUT as in
+ * ep_dispatch.  All argument checks of both calls apply, before anything
+ * is enqueued.
+ */
+ep_status_t ep_layout_dispatch(const void *idx, int idx_is_int64, int T,
+                               int k, int E, int R, const void *x, int H,
+                               int fp8, int32_t *cnt_e, int32_t *cnt_r,
+                               uint8_t *in_rank, int32_t *off_e,
+                               int32_t *off_r, int32_t *slot_pos,
+                               int32_t *recv_src, void *recv,
+                               float *recv_scale, void *ws, size_t ws_bytes,
+                               int num_sms, int32_t *d_err, void *stream);
+
+/*
  * ep_combine -- bring the expert outputs back to their tokens.
  *
  * DeepEP's combine (chinainews.com item, feature list; dataforcee.us

@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version():
-    assert ep.lib().ep_abi_version() == 2
+    assert ep.lib().ep_abi_version() == 3
 
 
 def test_workspace_sizes():
@@ -130,6 +130,36 @@ def test_rank_layout_workspace_sizes():
     assert ep.ep_rank_layout_workspace_bytes(4096, 8) == 0
     assert ep.ep_rank_layout_workspace_bytes(70000, 8) == ep.ep_layout_workspace_bytes(70000, 8, 8, 1)
     assert ep.ep_rank_layout_workspace_bytes(70000, 8) > 0
+
+
+def _layout_dispatch_call(**kw):
+    a = dict(idx=16, idx_is_int64=1, T=4, k=2, E=8, R=2, x=16, H=512, fp8=0, cnt_e=16,
+             cnt_r=16, in_rank=16, off_e=16, off_r=16, slot_pos=16, recv_src=16, recv=16,
+             recv_scale=None, ws=None, ws_bytes=0, num_sms=0, d_err=None, stream=None)
+    a.update(kw)
+    return ep.lib().ep_layout_dispatch(*a.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=-1), ep.EP_ERR_INVALID_ARG),
+    (dict(E=9), ep.EP_ERR_INVALID_ARG),                     # E % R != 0
+    (dict(k=33, E=64), ep.EP_ERR_UNSUPPORTED),
+    (dict(idx=None), ep.EP_ERR_INVALID_ARG),
+    (dict(slot_pos=None), ep.EP_ERR_INVALID_ARG),
+    (dict(x=None), ep.EP_ERR_INVALID_ARG),
+    (dict(x=24), ep.EP_ERR_INVALID_ARG),                    # x misaligned
+    (dict(recv=None), ep.EP_ERR_INVALID_ARG),
+    (dict(H=12), ep.EP_ERR_UNSUPPORTED),                    # H % 8
+    (dict(H=0), ep.EP_ERR_INVALID_ARG),
+    (dict(fp8=1, H=64, recv_scale=16), ep.EP_ERR_UNSUPPORTED),   # fp8, H % 128
+    (dict(fp8=1), ep.EP_ERR_INVALID_ARG),                   # fp8, no scales
+    (dict(num_sms=-1), ep.EP_ERR_INVALID_ARG),
+    (dict(d_err=2), ep.EP_ERR_INVALID_ARG),
+    (dict(T=65537, k=8, E=256, R=8), ep.EP_ERR_INVALID_ARG),     # two-kernel path, no ws
+])
+def test_layout_dispatch_rejects(kw, status):
+    assert _layout_dispatch_call(**kw) == status
+    assert ep.lib().ep_last_error_string().decode()
 
 
 def test_read_error_rejects_null():
