@@ -365,6 +365,7 @@ KERNEL_SOURCES = {
     "dispatch_bf16": ("dispatch.cu", "ep_internal.cuh"),
     "dispatch_fp8": ("dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
     "combine": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),
+    "layout_dispatch_fp8": ("layout_dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
 }
 
 
@@ -465,21 +466,24 @@ def bench_decode(ep, device, world, iters=200):
     stream.synchronize()
     us_stream = a.elapsed_time(b) * 1e3 / iters
 
-    def graph_us(fn):
-        """Device time of one replay of a CUDA graph holding fn's launches."""
+    def graph_us(fn, calls=1):
+        """Device time per call of fn, with `calls` back-to-back calls
+        captured in one CUDA graph and the graph replayed."""
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            fn()
+            for _ in range(calls):
+                fn()
+        reps = max(1, iters // calls)
         with torch.cuda.stream(stream):
-            for _ in range(20):
+            for _ in range(3):
                 g.replay()
             a.record(stream)
-            for _ in range(iters):
+            for _ in range(reps):
                 g.replay()
             b.record(stream)
         stream.synchronize()
         del g
-        return a.elapsed_time(b) * 1e3 / iters
+        return a.elapsed_time(b) * 1e3 / (reps * calls)
 
     c = cfg
 
@@ -497,6 +501,11 @@ def bench_decode(ep, device, world, iters=200):
 
     us_graph = graph_us(lambda: st.run(stream, fp8_only=True))
     us_fused = graph_us(fused_call)
+    # a decode step's graph holds more than one call: calls in sequence
+    # inside one graph overlap launch latency through programmatic
+    # dependent launch, and the graph's own launch is paid once
+    in_graph = {"unfused": graph_us(lambda: st.run(stream, fp8_only=True), calls=20),
+                "fused": graph_us(fused_call, calls=20)}
     # each kernel of the call alone, replayed from its own graph
     parts = {
         "layout": lambda: ep.ep_get_layout(st.idx, c.E, c.R, out=st.layout, ws=st.ws,
@@ -514,6 +523,7 @@ def bench_decode(ep, device, world, iters=200):
     us_stream = max_over_ranks(us_stream, world, device)
     us_graph = max_over_ranks(us_graph, world, device)
     us_fused = max_over_ranks(us_fused, world, device)
+    in_graph = {name: round(max_over_ranks(v, world, device), 2) for name, v in in_graph.items()}
     nb = decode_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R)
     return {"workload": "decode: T=128, H=7168, E=256/R=8, top-8, FP8 dispatch; "
                         "call = layout + FP8 dispatch + combine",
@@ -521,6 +531,7 @@ def bench_decode(ep, device, world, iters=200):
             "us_per_call_graph_fused": round(us_fused, 2),
             "fused": "ep_layout_dispatch (layout + FP8 dispatch, one kernel) + combine",
             "us_per_kernel_graph": part_us,
+            "us_per_call_in_graph_of_20": in_graph,
             "us_per_call_stream": round(us_stream, 2),
             "bytes_per_call": nb,
             "GB/s_graph": round(nb / (us_graph * 1e-6) / 1e9, 1),
@@ -683,6 +694,9 @@ def profile_kernel(args, device):
                                                d_err=st.d_err, stream=stream),
         "combine": lambda: ep.ep_combine(st.recv, st.layout.slot_pos, st.w, out=st.out,
                                          d_err=st.d_err, stream=stream),
+        "layout_dispatch_fp8": lambda: ep.ep_layout_dispatch(
+            st.idx, c.E, c.R, st.x, True, out=st.layout, recv=st.recv_q,
+            recv_scale=st.recv_s, ws=st.ws, d_err=st.d_err, stream=stream),
     }
     call = calls[args.profile]
     with torch.cuda.stream(stream):
@@ -719,7 +733,8 @@ def main():
     p.add_argument("--skip-dedup", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--reference-tokens", type=int, default=256)
-    p.add_argument("--profile", choices=("layout", "dispatch_bf16", "dispatch_fp8", "combine"),
+    p.add_argument("--profile", choices=("layout", "dispatch_bf16", "dispatch_fp8", "combine",
+                                         "layout_dispatch_fp8"),
                    help="run only this kernel (for profiler captures)")
     p.add_argument("--workload", choices=tuple(workloads.CONFIGS), default="prefill",
                    help="workload of --profile")

@@ -10,8 +10,13 @@
 // served by L2 after the first CTA reads them), with no CTA ever waiting on
 // another, then dispatches its own contiguous range of tokens and writes
 // the layout entries of those tokens; CTA 0 also writes the counts and
-// offsets.  The token rows are bulk-loaded (cp.async.bulk) before the
-// layout work starts, so the layout hides under the row loads.
+// offsets.
+//
+// Inside a CTA the work that does not need the layout runs beside it: the
+// token rows are bulk-loaded (cp.async.bulk) as the kernel starts, and
+// while warps 0..7 build the layout the other warps cast the first row to
+// FP8.  Once both are done, the receive rows are known and k threads issue
+// the bulk stores of the row, one receive row each.
 //
 // The layout in shared memory is one token bit set per expert: bit t % 32
 // of mask[e][t / 32] is set when token t chose expert e.  The receive row
@@ -30,21 +35,25 @@
 namespace ep {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / kWarp;
+constexpr int kLayoutThreads = 256;  // warps 0..7: the layout
+constexpr int kLayoutWarps = kLayoutThreads / kWarp;
+constexpr int kCastThreads = 512;    // warps 8..23: the first row's FP8 cast
+constexpr int kThreads = kLayoutThreads + kCastThreads;
 constexpr int kStages = 2;             // token rows in flight per CTA
 constexpr long kMaxSlots = 8192;       // T * k of the fused path
 constexpr long kMaxMaskBytes = 32768;  // E * ceil(T / 32) * 4
 constexpr int kMaxH = 16384;
+constexpr int kLayoutBarrier = 1;      // named barrier of the layout warps
 
 __host__ __device__ constexpr int align16(long b) { return static_cast<int>((b + 15) & ~15L); }
 
 // Byte offsets of the dynamic shared memory regions (host and device agree).
 struct SmemMap {
-  int in, out_q, out_s, mask, cnt, off, cnt_r, ids, total;
+  int in, out_q, out_s, mask, cnt, off, cnt_r, ids, rows, total;
 };
 
-__host__ __device__ inline SmemMap smem_map(int T, int k, int E, int R, int H, bool fp8) {
+__host__ __device__ inline SmemMap smem_map(int T, int k, int E, int R, int H, bool fp8,
+                                            int per_cta) {
   SmemMap m;
   const long W = (T + 31) / 32;
   int o = 0;
@@ -56,6 +65,7 @@ __host__ __device__ inline SmemMap smem_map(int T, int k, int E, int R, int H, b
   m.off = o;    o += align16(static_cast<long>(E + 1) * 4);
   m.cnt_r = o;  o += align16(static_cast<long>(R) * 4);
   m.ids = o;    o += align16(static_cast<long>(T) * k * 2);
+  m.rows = o;   o += align16(static_cast<long>(per_cta) * k * 4);  // this CTA's receive rows
   m.total = o;
   return m;
 }
@@ -63,6 +73,7 @@ __host__ __device__ inline SmemMap smem_map(int T, int k, int E, int R, int H, b
 struct FusedArgs {
   const void *idx;
   int T, k, E, R, G, H, W;
+  unsigned long long g_magic;  // ceil(2^32 / G): e / G == (e * g_magic) >> 32 for e < 1024
   const uint4 *x;
   int32_t *cnt_e, *cnt_r, *off_e, *off_r, *slot_pos, *recv_src;
   uint8_t *in_rank;
@@ -71,6 +82,10 @@ struct FusedArgs {
   int32_t *d_err;
   int per_cta;          // tokens per CTA
 };
+
+__device__ __forceinline__ void layout_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(kLayoutBarrier), "n"(kLayoutThreads) : "memory");
+}
 
 __device__ __forceinline__ int warp_incl_scan(int v) {
   const int lane = threadIdx.x & 31;
@@ -88,24 +103,24 @@ __device__ __forceinline__ int warp_sum(int v) {
   return v;
 }
 
-// out[0..n) = exclusive scan of in[0..n), out[n] = total, by the whole CTA
-// (each thread a contiguous run of ceil(n / kThreads) entries).
-__device__ void block_exclusive_scan(const int *in, int *out, int n, int *warp_tot) {
+// out[0..n) = exclusive scan of in[0..n), out[n] = total, by the layout
+// warps (each thread a contiguous run of ceil(n / kLayoutThreads) entries).
+__device__ void layout_exclusive_scan(const int *in, int *out, int n, int *warp_tot) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (n + kThreads - 1) / kThreads;
+  const int per = (n + kLayoutThreads - 1) / kLayoutThreads;
   const int b = min(n, tid * per), e = min(n, b + per);
   int local = 0;
   for (int q = b; q < e; ++q) local += in[q];
   const int incl = warp_incl_scan(local);
   if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
+  layout_sync();
   if (warp == 0) {
-    const int v = lane < kWarps ? warp_tot[lane] : 0;
+    const int v = lane < kLayoutWarps ? warp_tot[lane] : 0;
     const int iv = warp_incl_scan(v);
-    if (lane < kWarps) warp_tot[lane] = iv - v;
-    if (lane == kWarps - 1) out[n] = iv;
+    if (lane < kLayoutWarps) warp_tot[lane] = iv - v;
+    if (lane == kLayoutWarps - 1) out[n] = iv;
   }
-  __syncthreads();
+  layout_sync();
   int run = warp_tot[warp] + incl - local;
   for (int q = b; q < e; ++q) {
     out[q] = run;
@@ -113,43 +128,45 @@ __device__ void block_exclusive_scan(const int *in, int *out, int n, int *warp_t
   }
 }
 
+// e4m3 codes and scales of one bf16 row (smem) into the output stage, by
+// the `nthreads` threads numbered ctid = 0..nthreads-1 (a multiple of 32):
+// a half-warp per 128-channel block; whole warps share the loop bound
+// because H / 8 is a multiple of 64.
+__device__ __forceinline__ void cast_row(const uint4 *xin, uint2 *qo, float *so, int H, int ctid,
+                                         int nthreads) {
+  for (int v = ctid; v < (H >> 3); v += nthreads) {
+    float sc;
+    qo[v] = quantize_block_lane(xin[v], &sc);
+    if ((ctid & 15) == 0) so[v >> 4] = sc;
+  }
+}
+
 template <typename IdT, bool kFp8>
 __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(const FusedArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const SmemMap sm = smem_map(a.T, a.k, a.E, a.R, a.H, kFp8);
+  const SmemMap sm = smem_map(a.T, a.k, a.E, a.R, a.H, kFp8, a.per_cta);
   unsigned char *in_buf = smem + sm.in;
-  unsigned char *out_q = smem + sm.out_q;
+  uint2 *out_q = reinterpret_cast<uint2 *>(smem + sm.out_q);
   float *out_s = reinterpret_cast<float *>(smem + sm.out_s);
   unsigned *mask = reinterpret_cast<unsigned *>(smem + sm.mask);
   int *cnt = reinterpret_cast<int *>(smem + sm.cnt);
   int *off = reinterpret_cast<int *>(smem + sm.off);
   int *cnt_r = reinterpret_cast<int *>(smem + sm.cnt_r);
   int16_t *ids = reinterpret_cast<int16_t *>(smem + sm.ids);
+  int *rows = reinterpret_cast<int *>(smem + sm.rows);  // [per_cta][k]
   __shared__ __align__(8) uint64_t full[kStages];
-  __shared__ int rows[2][EP_MAX_K];
-  __shared__ int warp_tot[kWarps];
+  __shared__ int warp_tot[kLayoutWarps];
   __shared__ int dup;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int T = a.T, k = a.k, E = a.E, R = a.R, G = a.G, H = a.H, W = a.W;
-  const long N = static_cast<long>(T) * k;
+  const int N = T * k;
   const int first = blockIdx.x * a.per_cta;
   const int n_mine = max(0, min(T, first + a.per_cta) - first);
   const int in_bytes = 2 * H;
   const bool lead = blockIdx.x == 0;
 
   pdl_trigger();
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
-    mbar_init_fence();
-    dup = 0;
-  }
-  for (int q = tid; q < E * W; q += kThreads) mask[q] = 0u;
-  for (int q = tid; q < E; q += kThreads) cnt[q] = 0;
-  for (int q = tid; q < R; q += kThreads) cnt_r[q] = 0;
-  __syncthreads();
-  pdl_wait();  // ids and rows come from the previous kernel on the stream
-
   // thread 0: token first + i -> input stage i % kStages
   auto issue = [&](int i) {
     const int s = i % kStages;
@@ -157,177 +174,222 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(const FusedAr
     bulk_load(in_buf + s * in_bytes, a.x + static_cast<long>(first + i) * (H >> 3), in_bytes,
               &full[s]);
   };
-  if (tid == 0)
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    mbar_init_fence();
+    dup = 0;
+    pdl_wait();  // rows and ids come from the previous kernel on the stream
     for (int i = 0; i < min(kStages, n_mine); ++i) issue(i);
+  }
+  for (int q = tid; q < E * W; q += kThreads) mask[q] = 0u;
+  for (int q = tid; q < E; q += kThreads) cnt[q] = 0;
+  for (int q = tid; q < R; q += kThreads) cnt_r[q] = 0;
+  pdl_wait();
+  __syncthreads();
 
-  // 1. ids -> per-expert token sets and slot counts (bad ids reported once)
-  const IdT *idx = static_cast<const IdT *>(a.idx);
-  constexpr int kBatch = 4;
-  for (long base = 0; base < N; base += kBatch * kThreads) {
-    long long v[kBatch];
+  bool ok = true;  // this thread's row wait did not time out
+  if (tid < kLayoutThreads) {
+    // ---- the layout (warps 0..7) ----
+    // 1. ids -> per-expert token sets and slot counts (bad ids reported once)
+    const IdT *idx = static_cast<const IdT *>(a.idx);
+    constexpr int kBatch = 4;
+    for (int base = 0; base < N; base += kBatch * kLayoutThreads) {
+      long long v[kBatch];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const long i = base + u * kThreads + tid;
-      v[u] = i < N ? static_cast<long long>(idx[i]) : -1;
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const long i = base + u * kThreads + tid;
-      if (i >= N) continue;
-      int e = -1;
-      if (v[u] >= 0 && v[u] < E)
-        e = static_cast<int>(v[u]);
-      else if (v[u] != -1 && lead && a.d_err != nullptr)
-        atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_INDEX);
-      ids[i] = static_cast<int16_t>(e);
-      if (e >= 0) {
-        const int t = static_cast<int>(i / k);
-        const unsigned bit = 1u << (t & 31);
-        if (atomicOr(&mask[e * W + (t >> 5)], bit) & bit) dup = 1;
-        atomicAdd(&cnt[e], 1);
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = base + u * kLayoutThreads + tid;
+        v[u] = i < N ? static_cast<long long>(idx[i]) : -1;
       }
-    }
-  }
-  __syncthreads();
-
-  // 2. offsets; CTA 0 also counts the tokens of each rank
-  block_exclusive_scan(cnt, off, E, warp_tot);
-  if (lead) {
-    for (int q = tid; q < R * W; q += kThreads) {
-      const int r = q / W, w = q - r * W;
-      unsigned m = 0u;
-      for (int g = 0; g < G; ++g) m |= mask[(r * G + g) * W + w];
-      if (m != 0u) atomicAdd(&cnt_r[r], __popc(m));
-    }
-  }
-  __syncthreads();
-  const int n_eff = off[E];
-  if (lead) {
-    for (int q = tid; q < E; q += kThreads) {
-      a.cnt_e[q] = cnt[q];
-      a.off_e[q] = off[q];
-    }
-    if (tid == 0) a.off_e[E] = n_eff;
-    if (warp == kWarps - 1) {  // R <= 64
-      int carry = 0;
-      for (int b = 0; b < R; b += 32) {
-        const int r = b + lane;
-        const int c = r < R ? cnt_r[r] : 0;
-        const int incl = warp_incl_scan(c);
-        if (r < R) {
-          a.cnt_r[r] = c;
-          a.off_r[r] = carry + incl - c;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = base + u * kLayoutThreads + tid;
+        if (i >= N) continue;
+        int e = -1;
+        if (v[u] >= 0 && v[u] < E)
+          e = static_cast<int>(v[u]);
+        else if (v[u] != -1 && lead && a.d_err != nullptr)
+          atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_INDEX);
+        ids[i] = static_cast<int16_t>(e);
+        if (e >= 0) {
+          const int t = i / k;
+          const unsigned bit = 1u << (t & 31);
+          if (atomicOr(&mask[e * W + (t >> 5)], bit) & bit) dup = 1;
+          atomicAdd(&cnt[e], 1);
         }
-        carry += __shfl_sync(0xffffffffu, incl, 31);
       }
-      if (lane == 0) a.off_r[R] = carry;
     }
-  }
-  // receive rows no slot points at
-  for (long r = n_eff + static_cast<long>(blockIdx.x) * kThreads + tid; r < N;
-       r += static_cast<long>(gridDim.x) * kThreads)
-    a.recv_src[r] = -1;
+    layout_sync();
 
-  // 3. this CTA's tokens: rows and layout entries, then the dispatch
-  int i = 0;
-  bool timed_out = false;
-  for (; i < n_mine; ++i) {
-    const int t = first + i;
-    const int s = i % kStages;
-    const int rb = i & 1;
-    for (int j = warp; j < k; j += kWarps) {  // a warp per slot
-      const int e = ids[t * k + j];
-      int before = 0;
-      if (e >= 0) {
+    // 2. offsets; CTA 0 also counts the tokens of each rank (a token's ranks
+    //    as a bit mask over its ids, R <= 64)
+    if (lead) {
+      for (int t = tid; t < T; t += kLayoutThreads) {
+        unsigned long long rm = 0ull;
+        for (int j = 0; j < k; ++j) {
+          const int e = ids[t * k + j];
+          if (e >= 0) rm |= 1ull << ((static_cast<unsigned long long>(e) * a.g_magic) >> 32);
+        }
+        while (rm != 0ull) {
+          atomicAdd(&cnt_r[__ffsll(static_cast<long long>(rm)) - 1], 1);
+          rm &= rm - 1ull;
+        }
+      }
+    }
+    layout_exclusive_scan(cnt, off, E, warp_tot);
+    layout_sync();
+    const int n_eff = off[E];
+    if (lead) {
+      for (int q = tid; q < E; q += kLayoutThreads) {
+        a.cnt_e[q] = cnt[q];
+        a.off_e[q] = off[q];
+      }
+      if (tid == 0) a.off_e[E] = n_eff;
+      if (warp == kLayoutWarps - 1) {
+        int carry = 0;
+        for (int b = 0; b < R; b += 32) {
+          const int r = b + lane;
+          const int c = r < R ? cnt_r[r] : 0;
+          const int incl = warp_incl_scan(c);
+          if (r < R) {
+            a.cnt_r[r] = c;
+            a.off_r[r] = carry + incl - c;
+          }
+          carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) a.off_r[R] = carry;
+      }
+    }
+    // receive rows no slot points at
+    for (int r = n_eff + blockIdx.x * kLayoutThreads + tid; r < N;
+         r += gridDim.x * kLayoutThreads)
+      a.recv_src[r] = -1;
+
+    // 3. receive rows of this CTA's slots: a thread per slot when the token
+    //    sets are short (<= 4 words), else a warp per slot
+    const int n_slots = n_mine * k;
+    const int f0 = first * k;
+    auto place = [&](int q, int before) {
+      const int e = ids[f0 + q];
+      const int row = e >= 0 ? off[e] + before : -1;
+      rows[q] = row;
+      a.slot_pos[f0 + q] = row;
+      if (row >= 0) a.recv_src[row] = first + q / k;
+    };
+    if (!dup && W <= 4) {
+      for (int q = tid; q < n_slots; q += kLayoutThreads) {
+        const int e = ids[f0 + q];
         int c = 0;
-        if (!dup) {  // tokens before t that chose e
+        if (e >= 0) {
+          const int t = first + q / k;
           const unsigned *me = mask + e * W;
-          const int wt = t >> 5;
-          for (int w = lane; w < wt; w += 32) c += __popc(me[w]);
-          if (lane == 0) c += __popc(me[wt] & ((1u << (t & 31)) - 1u));
-        } else {  // slots before (t, j) in token-major order with expert e
-          const int flat = t * k + j;
-          for (int q = lane; q < flat; q += 32) c += ids[q] == e;
+          for (int w = 0; w < (t >> 5); ++w) c += __popc(me[w]);
+          c += __popc(me[t >> 5] & ((1u << (t & 31)) - 1u));
         }
-        before = warp_sum(c);
+        place(q, c);
       }
-      if (lane == 0) {
-        const int row = e >= 0 ? off[e] + before : -1;
-        rows[rb][j] = row;
-        a.slot_pos[static_cast<long>(t) * k + j] = row;
-        if (row >= 0) a.recv_src[row] = t;
+    } else {
+      for (int q = warp; q < n_slots; q += kLayoutWarps) {
+        const int e = ids[f0 + q];
+        int c = 0;
+        if (e >= 0) {
+          if (!dup) {  // tokens before t that chose e
+            const int t = first + q / k;
+            const unsigned *me = mask + e * W;
+            const int wt = t >> 5;
+            for (int w = lane; w < wt; w += 32) c += __popc(me[w]);
+            if (lane == 0) c += __popc(me[wt] & ((1u << (t & 31)) - 1u));
+          } else {  // slots before this one in token-major order with expert e
+            for (int p = lane; p < f0 + q; p += 32) c += ids[p] == e;
+          }
+          c = warp_sum(c);
+        }
+        if (lane == 0) place(q, c);
       }
     }
-    for (int r = tid; r < R; r += kThreads) {
+    // token-in-rank entries of this CTA's tokens
+    for (int q = tid; q < n_mine * R; q += kLayoutThreads) {
+      const int t = first + q / R, r = q - (q / R) * R;
       int in = 0;
-      for (int j = 0; j < k; ++j) {
-        const int e = ids[t * k + j];
-        in |= e >= 0 && e / G == r;
-      }
+      for (int j = 0; j < k; ++j)
+        in |= static_cast<unsigned>(ids[t * k + j] - r * G) < static_cast<unsigned>(G);
       a.in_rank[static_cast<long>(t) * R + r] = static_cast<uint8_t>(in);
     }
-    if (kFp8 && tid == 0) bulk_wait_read<0>();  // the previous token's stores left out_q
-    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1));
-    if (__syncthreads_or(!ok)) {
-      timed_out = true;
-      break;
-    }
-    if (kFp8) {
-      const uint4 *xin = reinterpret_cast<const uint4 *>(in_buf + s * in_bytes);
-      uint2 *qo = reinterpret_cast<uint2 *>(out_q);
-      // a half-warp per 128-channel block; whole warps share the loop bound
-      // because H / 8 is a multiple of 64
-      for (int v = tid; v < (H >> 3); v += kThreads) {
-        float sc;
-        qo[v] = quantize_block_lane(xin[v], &sc);
-        if ((tid & 15) == 0) out_s[v >> 4] = sc;
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (tid == 0) {
-        const int nb = H >> 7;
-        for (int j = 0; j < k; ++j) {
-          const int row = rows[rb][j];
-          if (row < 0) continue;
-          bulk_store(a.recv + static_cast<long>(row) * H, out_q, H);
-          bulk_store(a.recv_scale + static_cast<long>(row) * nb, out_s, 4 * nb);
-        }
-        bulk_commit();
-        if (i + kStages < n_mine) issue(i + kStages);  // stage s was read by the cast only
-      }
-    } else if (tid == 0) {
-      for (int j = 0; j < k; ++j) {
-        const int row = rows[rb][j];
-        if (row < 0) continue;
-        bulk_store(a.recv + static_cast<long>(row) * in_bytes, in_buf + s * in_bytes, in_bytes);
-      }
-      bulk_commit();
-      if (i + kStages < n_mine) {
-        bulk_wait_read<0>();  // the stores above have read stage s
-        issue(i + kStages);
-      }
+  } else if (n_mine > 0) {
+    // ---- the first row (warps 8..): wait for it, cast it to FP8 ----
+    ok = mbar_wait_bounded(&full[0], 0u);
+    if (kFp8 && ok) {
+      cast_row(reinterpret_cast<const uint4 *>(in_buf), out_q, out_s, H, tid - kLayoutThreads,
+               kCastThreads);
+      fence_proxy_async_smem();  // the stage's generic writes before the bulk reads
     }
   }
-  if (tid == 0) {
-    if (timed_out) {
-      if (a.d_err != nullptr) atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_TIMEOUT);
-      // let the row loads still in flight land before the CTA's memory goes away
-      for (int q = i; q < min(n_mine, i + kStages); ++q)
-        mbar_wait_bounded(&full[q % kStages], static_cast<unsigned>((q / kStages) & 1));
+  bool timed_out = __syncthreads_or(!ok);
+
+  // 4. per token: (after the first) wait for its row and cast it, then k
+  //    threads store it, one receive row each
+  int i = 0;
+  for (; i < n_mine && !timed_out; ++i) {
+    const int s = i % kStages;
+    if (i > 0) {
+      ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1));
+      if (__syncthreads_or(!ok)) {
+        timed_out = true;
+        break;
+      }
+      if (kFp8) {
+        cast_row(reinterpret_cast<const uint4 *>(in_buf + s * in_bytes), out_q, out_s, H, tid,
+                 kThreads);
+        fence_proxy_async_smem();
+        __syncthreads();
+      }
     }
-    bulk_wait<0>();
+    if (tid < k) {
+      // bf16: the stores read the bulk-loaded stage itself; their issuer
+      // observes its completion (already passed, so this returns at once)
+      if (!kFp8) mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1));
+      const int row = rows[i * k + tid];
+      if (row >= 0) {
+        if (kFp8) {
+          const int nb = H >> 7;
+          bulk_store(a.recv + static_cast<long>(row) * H, out_q, H);
+          bulk_store(a.recv_scale + static_cast<long>(row) * nb, out_s, 4 * nb);
+        } else {
+          bulk_store(a.recv + static_cast<long>(row) * in_bytes, in_buf + s * in_bytes, in_bytes);
+        }
+      }
+      bulk_commit();
+    }
+    if (i + 1 < n_mine) {
+      // the output stage (FP8) and input stage s (both) are read by the
+      // stores: wait for that before they are overwritten
+      if (tid < k) bulk_wait_read<0>();
+      __syncthreads();
+      if (tid == 0 && i + kStages < n_mine) issue(i + kStages);
+    }
+  }
+  if (tid < k) bulk_wait<0>();
+  if (tid == 0 && timed_out) {
+    if (a.d_err != nullptr) atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_TIMEOUT);
+    // let the row loads still in flight land before the CTA's memory goes away
+    for (int q = i; q < min(n_mine, i + kStages); ++q)
+      mbar_wait_bounded(&full[q % kStages], static_cast<unsigned>((q / kStages) & 1));
   }
 }
 
 template <typename IdT, bool kFp8>
 cudaError_t launch_fused(const FusedArgs &base, int num_sms, cudaStream_t s) {
   auto kern = layout_dispatch_kernel<IdT, kFp8>;
-  const int smem = smem_map(base.T, base.k, base.E, base.R, base.H, kFp8).total;
+  // shared memory sized for ceil(T / SMs) tokens per CTA, which bounds the
+  // tokens of a CTA below (at least one CTA per SM fits)
+  const int sms = num_sms > 0 ? num_sms : device_sm_count();
+  const int per_cta_max = (base.T + sms - 1) / sms;
+  const int smem =
+      smem_map(base.T, base.k, base.E, base.R, base.H, kFp8, per_cta_max).total;
   cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
   if (err != cudaSuccess) return err;
   // a CTA per token, capped at the CTAs that fit at once; no CTA left empty
   const long cap = persistent_grid(reinterpret_cast<const void *>(kern), kThreads, smem,
-                                   static_cast<long>(base.T) * kWarps, num_sms);
+                                   static_cast<long>(base.T) * (kThreads / kWarp), num_sms);
   FusedArgs a = base;
   a.per_cta = static_cast<int>((base.T + cap - 1) / cap);
   const int grid = (base.T + a.per_cta - 1) / a.per_cta;
@@ -355,6 +417,7 @@ cudaError_t launch_layout_dispatch(const LayoutArgs &la, const void *x, int H, b
   a.E = la.E;
   a.R = la.R;
   a.G = la.E / la.R;
+  a.g_magic = ((1ull << 32) + a.G - 1) / a.G;
   a.H = H;
   a.W = (la.T + 31) / 32;
   a.x = static_cast<const uint4 *>(x);
