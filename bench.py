@@ -351,6 +351,8 @@ def bench_ours(args, world, rank, device):
         result["decode"] = bench_decode(ep, device, world)
     if not args.skip_dedup:
         result["rank_dedup"] = bench_rank_dedup(ep, st, cfg, device, world)
+    if not args.skip_overlap:
+        result["sm_budget_overlap"] = bench_overlap(ep, st, cfg, device, world)
     if not args.skip_e2e:
         result["e2e"] = bench_e2e(ep, cfg, batch, device, args, world, total_bytes)
     if world == 1 and rank == 0 and not args.skip_cpu:
@@ -445,6 +447,87 @@ def bench_rank_dedup(ep, st, cfg, device, world, iters=20):
                             world, device)
         res[name] = {"us": round(us, 2), "bytes": nbytes,
                      "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)}
+    return res
+
+
+OVERLAP_GEMM = (4096, 7168, 2048)   # M, K, N of the stand-in expert GEMM
+OVERLAP_SMS = (16, 32, 64, 148)
+
+
+def bench_overlap(ep, st, cfg, device, world, reps=10):
+    """SM-budgeted dispatch and combine beside a GEMM on another stream.
+
+    DeepEP's normal kernels run on a fixed budget of SMs so that the rest
+    can compute at the same time (frogred8 blog, "deepEP optimization",
+    third method: the SM count is a parameter).  The GEMM stands in for the
+    expert computation (cuBLAS through torch.matmul, bf16, M x K @ K x N).
+    For each SM budget S: the bf16 dispatch (or combine) alone with
+    num_sms=S, the GEMM alone, and both launched together on two streams;
+    `both_us` runs from a common start event until both streams are done
+    (L2 flushed before each trial).  `overlap` = (alone + gemm) / both:
+    1 means no overlap, 2 perfect overlap of equal halves."""
+    M, K, N = OVERLAP_GEMM
+    gen = torch.Generator(device=device).manual_seed(7)
+    A = torch.randn((M, K), device=device, dtype=torch.bfloat16, generator=gen)
+    B = torch.randn((K, N), device=device, dtype=torch.bfloat16, generator=gen)
+    Cm = torch.empty((M, N), device=device, dtype=torch.bfloat16)
+    s_comm = torch.cuda.Stream(device)
+    s_comp = torch.cuda.Stream(device)
+    flush = L2Flush(device)
+    with torch.cuda.stream(s_comm):
+        st.run(s_comm)   # a valid layout and receive buffer
+    s_comm.synchronize()
+
+    def gemm():
+        torch.matmul(A, B, out=Cm)
+
+    ops = {
+        "dispatch_bf16": lambda S: ep.ep_dispatch(st.x, st.layout.slot_pos, recv=st.recv,
+                                                  num_sms=S, d_err=st.d_err, stream=s_comm),
+        "combine": lambda S: ep.ep_combine(st.recv, st.layout.slot_pos, st.w, out=st.out,
+                                           num_sms=S, d_err=st.d_err, stream=s_comm),
+    }
+
+    def trial(comm, comp):
+        """Device microseconds from a common start until both streams end."""
+        torch.cuda.synchronize(device)
+        flush()
+        torch.cuda.synchronize(device)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(s_comm)
+        s_comp.wait_event(ev[0])
+        if comm is not None:
+            with torch.cuda.stream(s_comm):
+                comm()
+        if comp is not None:
+            with torch.cuda.stream(s_comp):
+                comp()
+        ev[1].record(s_comm)
+        ev[2].record(s_comp)
+        torch.cuda.synchronize(device)
+        return max(ev[0].elapsed_time(ev[1]), ev[0].elapsed_time(ev[2])) * 1e3
+
+    def median(fn):
+        fn()
+        return statistics.median(fn() for _ in range(reps))
+
+    gemm_us = median(lambda: trial(None, gemm))
+    res = {"gemm": {"mkn": [M, K, N], "us": round(max_over_ranks(gemm_us, world, device), 2),
+                    "TFLOP/s": round(2 * M * K * N / (gemm_us * 1e-6) / 1e12, 1)},
+           "note": "both_us = dispatch or combine and the GEMM on two streams at once"}
+    for name, op in ops.items():
+        rows = []
+        for S in OVERLAP_SMS:
+            alone = median(lambda: trial(lambda: op(S), None))
+            both = median(lambda: trial(lambda: op(S), gemm))
+            alone = max_over_ranks(alone, world, device)
+            both = max_over_ranks(both, world, device)
+            rows.append({"num_sms": S, "alone_us": round(alone, 2), "both_us": round(both, 2),
+                         "serial_us": round(alone + gemm_us, 2),
+                         "overlap": round((alone + gemm_us) / both, 3)})
+        res[name] = rows
+    if ep.ep_read_error(st.d_err, s_comm) != 0:
+        raise RuntimeError("the device reported an error in the overlap runs")
     return res
 
 
@@ -731,6 +814,7 @@ def main():
     p.add_argument("--skip-e2e", action="store_true")
     p.add_argument("--skip-cpu", action="store_true")
     p.add_argument("--skip-dedup", action="store_true")
+    p.add_argument("--skip-overlap", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--reference-tokens", type=int, default=256)
     p.add_argument("--profile", choices=("layout", "dispatch_bf16", "dispatch_fp8", "combine",

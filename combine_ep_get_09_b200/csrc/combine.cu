@@ -59,66 +59,65 @@ __global__ void __launch_bounds__(kChunkVec)
   __shared__ __align__(8) uint64_t full[kStages];
   __shared__ int stage_row[kStages][kBulkMaxK];
   __shared__ float stage_w[kStages][kBulkMaxK];
-  __shared__ int timed_out;
 
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int nchunks = (Hv + kChunkVec - 1) / kChunkVec;
   const long items = static_cast<long>(T) * nchunks;
-  const long per_cta = (items + gridDim.x - 1) / gridDim.x;
-  const long first = min(items, static_cast<long>(blockIdx.x) * per_cta);
-  const long n_mine = min(items, first + per_cta) - first;
+  // CTA b walks items [items * b / grid, items * (b + 1) / grid): the
+  // shares differ by at most one item
+  const long first = items * blockIdx.x / gridDim.x;
+  const long n_mine = items * (blockIdx.x + 1) / gridDim.x - first;
 
   pdl_trigger();
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    // every lane of warp 0 arrives once per phase (see issue)
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], kWarp);
     mbar_init_fence();
-    timed_out = 0;
   }
   __syncthreads();
   pdl_wait();
 
-  // thread 0: gather item i's slot rows into stage i % kStages
+  // warp 0: lane j < k gathers the chunk of item i's slot row j into stage
+  // i % kStages.  Each lane announces its own bytes with its arrival, so
+  // the row indices and weights it leaves in shared memory are published
+  // with it; dropped slots arrive with 0 bytes.
   auto issue = [&](long i) {
     const long it = first + i;
     const int s = static_cast<int>(i % kStages);
     const int t = static_cast<int>(it / nchunks);
     const int v0 = static_cast<int>(it % nchunks) * kChunkVec;
     const unsigned bytes = static_cast<unsigned>(min(kChunkVec, Hv - v0)) * 16u;
-    int rows[kBulkMaxK];
-    int n_valid = 0;
-#pragma unroll
-    for (int j = 0; j < kBulkMaxK; ++j) {
-      int r = -1;
-      float wj = 0.0f;
-      if (j < k) {
-        r = __ldg(slot_pos + static_cast<long>(t) * k + j);
-        wj = w != nullptr ? __ldg(w + static_cast<long>(t) * k + j) : 1.0f;
-        if (r < 0 || r >= n_rows) r = -1;
-      }
-      rows[j] = r;
-      stage_row[s][j] = r;
-      stage_w[s][j] = wj;
-      n_valid += r >= 0;
+    int r = -1;
+    if (lane < k) {
+      r = __ldg(slot_pos + static_cast<long>(t) * k + lane);
+      const float wj = w != nullptr ? __ldg(w + static_cast<long>(t) * k + lane) : 1.0f;
+      if (r < 0 || r >= n_rows) r = -1;
+      stage_row[s][lane] = r;
+      stage_w[s][lane] = wj;
+    } else if (lane < kBulkMaxK) {
+      stage_row[s][lane] = -1;
     }
-    // the arrival publishes stage_row / stage_w (release) with the byte count
-    mbar_arrive_expect_tx(&full[s], n_valid * bytes);
-#pragma unroll
-    for (int j = 0; j < kBulkMaxK; ++j)
-      if (rows[j] >= 0)
-        bulk_load(stage_buf + (s * kBulkMaxK + j) * kChunkVec,
-                  y + static_cast<long>(rows[j]) * Hv + v0, bytes, &full[s]);
+    mbar_arrive_expect_tx(&full[s], r >= 0 ? bytes : 0u);
+    if (r >= 0)
+      bulk_load(stage_buf + (s * kBulkMaxK + lane) * kChunkVec, y + static_cast<long>(r) * Hv + v0,
+                bytes, &full[s]);
   };
 
-  if (tid == 0)
+  if (tid < kWarp)
     for (long i = 0; i < min(static_cast<long>(kStages), n_mine); ++i) issue(i);
 
   long i = 0;
+  bool timed_out = false;
   for (; i < n_mine; ++i) {
     const int s = static_cast<int>(i % kStages);
     const long it = first + i;
     const int t = static_cast<int>(it / nchunks);
     const int v0 = static_cast<int>(it % nchunks) * kChunkVec;
-    if (!mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1))) timed_out = 1;
+    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1));
+    if (__syncthreads_or(!ok)) {
+      timed_out = true;
+      break;
+    }
     if (tid < Hv - v0) {
       float acc[8];
 #pragma unroll
@@ -130,13 +129,12 @@ __global__ void __launch_bounds__(kChunkVec)
       st_stream_v4(out + static_cast<long>(t) * Hv + v0 + tid, to_bf16x8(acc));
     }
     __syncthreads();  // stage s fully read
-    if (timed_out) break;
-    if (tid == 0 && i + kStages < n_mine) issue(i + kStages);
+    if (tid < kWarp && i + kStages < n_mine) issue(i + kStages);
   }
   if (timed_out && tid == 0) {
     if (d_err != nullptr) atomicExch(reinterpret_cast<int *>(d_err), EP_ERR_TIMEOUT);
     // let the copies still in flight land before the CTA's memory goes away
-    for (long q = i + 1; q < min(n_mine, i + kStages); ++q)
+    for (long q = i; q < min(n_mine, i + kStages); ++q)
       mbar_wait_bounded(&full[q % kStages], static_cast<unsigned>((q / kStages) & 1));
   }
 }

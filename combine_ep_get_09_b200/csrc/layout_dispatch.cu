@@ -18,6 +18,19 @@
 // FP8.  Once both are done, the receive rows are known and k threads issue
 // the bulk stores of the row, one receive row each.
 //
+// Two kernels:
+//  * layout_dispatch_token_kernel (T + 1 CTAs fit on the GPU at once, e.g.
+//    a 128-token decode step): CTA b < T owns token b only.  The receive
+//    row of its slot (b, j) with expert e is the number of kept slots whose
+//    (expert, flat slot index) key is smaller than (e, b*k + j): expert-
+//    major, token-major inside an expert -- the stable order of the unfused
+//    layout, duplicates included.  The CTA counts those keys over all ids
+//    (each thread a strided share, a warp-wide sum, one shared atomic per
+//    warp and slot), so it needs no table, no scan and no zeroing; CTA T
+//    alone builds the per-expert and per-rank counts and offsets.
+//  * layout_dispatch_kernel (larger batches): CTAs own contiguous token
+//    ranges and each builds the token-set table below.
+//
 // The layout in shared memory is one token bit set per expert: bit t % 32
 // of mask[e][t / 32] is set when token t chose expert e.  The receive row
 // of slot (t, j) with expert e is off_e[e] + (tokens before t that chose e),
@@ -376,8 +389,249 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(const FusedAr
   }
 }
 
+// ------------------------------------------------ one token per CTA
+
+constexpr int kTokThreads = 512;
+constexpr int kTokWarps = kTokThreads / kWarp;
+constexpr int kTokIdBatch = 4;  // ids per thread loaded before the cast
+
+__host__ __device__ inline SmemMap token_smem_map(int T, int k, int E, int R, int H, bool fp8) {
+  SmemMap m;
+  int o = 0;
+  m.in = o;     o += 2 * H;
+  m.out_q = o;  o += fp8 ? H : 0;
+  m.out_s = o;  o += fp8 ? H / 32 : 0;
+  m.mask = o;   // unused
+  m.cnt = o;    o += align16(static_cast<long>(E) * 4);
+  m.off = o;    o += align16(static_cast<long>(E + 1) * 4);
+  m.cnt_r = o;  o += align16(static_cast<long>(R) * 4);
+  m.ids = o;    o += align16(static_cast<long>(T) * k * 2);
+  m.rows = o;
+  m.total = o;
+  return m;
+}
+
+__device__ __forceinline__ int valid_id(long long v, int E) {
+  return v >= 0 && v < E ? static_cast<int>(v) : -1;
+}
+
+// out[0..n) = exclusive scan of in[0..n), out[n] = total, by all
+// kTokThreads threads of the CTA.
+__device__ void token_cta_exclusive_scan(const int *in, int *out, int n, int *warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n + kTokThreads - 1) / kTokThreads;
+  const int b = min(n, tid * per), e = min(n, b + per);
+  int local = 0;
+  for (int q = b; q < e; ++q) local += in[q];
+  const int incl = warp_incl_scan(local);
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < kTokWarps ? warp_tot[lane] : 0;
+    const int iv = warp_incl_scan(v);
+    if (lane < kTokWarps) warp_tot[lane] = iv - v;
+    if (lane == kTokWarps - 1) out[n] = iv;
+  }
+  __syncthreads();
+  int run = warp_tot[warp] + incl - local;
+  for (int q = b; q < e; ++q) {
+    out[q] = run;
+    run += in[q];
+  }
+}
+
+template <typename IdT, bool kFp8>
+__global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(const FusedArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const SmemMap sm = token_smem_map(a.T, a.k, a.E, a.R, a.H, kFp8);
+  unsigned char *in_buf = smem + sm.in;
+  uint2 *out_q = reinterpret_cast<uint2 *>(smem + sm.out_q);
+  float *out_s = reinterpret_cast<float *>(smem + sm.out_s);
+  int *cnt = reinterpret_cast<int *>(smem + sm.cnt);
+  int *off = reinterpret_cast<int *>(smem + sm.off);
+  int *cnt_r = reinterpret_cast<int *>(smem + sm.cnt_r);
+  int16_t *ids = reinterpret_cast<int16_t *>(smem + sm.ids);
+  __shared__ __align__(8) uint64_t full;
+  __shared__ int rank_sm[EP_MAX_K];
+  __shared__ int warp_tot[kTokWarps];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = a.T, k = a.k, E = a.E, R = a.R, G = a.G, H = a.H;
+  const int N = T * k;
+  const int t = blockIdx.x;          // this CTA's token (t == T: the counts CTA)
+  const bool counts_cta = t == T;
+  const IdT *idx = static_cast<const IdT *>(a.idx);
+
+  pdl_trigger();
+  if (tid == 0 && !counts_cta) {
+    mbar_init(&full, 1);
+    mbar_init_fence();
+  }
+  if (counts_cta) {
+    for (int q = tid; q < E; q += kTokThreads) cnt[q] = 0;
+    for (int q = tid; q < R; q += kTokThreads) cnt_r[q] = 0;
+  } else if (tid < EP_MAX_K) {
+    rank_sm[tid] = 0;
+  }
+  __syncthreads();  // barrier initialised and counters zeroed before use
+  pdl_wait();       // ids and the row come from the previous kernel on the stream
+  if (tid == 0 && !counts_cta) {
+    mbar_arrive_expect_tx(&full, 2 * H);
+    bulk_load(in_buf, a.x + static_cast<long>(t) * (H >> 3), 2 * H, &full);
+  }
+
+  // 1. ids into shared memory (validated: -1 for dropped and bad slots);
+  //    a dispatch CTA casts its row to FP8 while the first batch is in flight
+  long long v[kTokIdBatch];
+#pragma unroll
+  for (int u = 0; u < kTokIdBatch; ++u) {
+    const int q = u * kTokThreads + tid;
+    v[u] = q < N ? static_cast<long long>(idx[q]) : -1;
+  }
+  bool ok = true;
+  if (!counts_cta) {
+    ok = mbar_wait_bounded(&full, 0u);
+    if (kFp8 && ok) {
+      cast_row(reinterpret_cast<const uint4 *>(in_buf), out_q, out_s, H, tid, kTokThreads);
+      fence_proxy_async_smem();  // the stage's generic writes before the bulk reads
+    }
+  }
+  auto take = [&](int q, long long raw) {
+    const int e = valid_id(raw, E);
+    ids[q] = static_cast<int16_t>(e);
+    if (counts_cta) {
+      if (e >= 0)
+        atomicAdd(&cnt[e], 1);
+      else if (raw != -1 && a.d_err != nullptr)
+        atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_INDEX);
+    }
+  };
+#pragma unroll
+  for (int u = 0; u < kTokIdBatch; ++u) {
+    const int q = u * kTokThreads + tid;
+    if (q < N) take(q, v[u]);
+  }
+  for (int q = kTokIdBatch * kTokThreads + tid; q < N; q += kTokThreads)
+    take(q, static_cast<long long>(idx[q]));
+  if (__syncthreads_or(!ok)) {
+    if (tid == 0) {
+      if (a.d_err != nullptr) atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_TIMEOUT);
+      mbar_wait_bounded(&full, 0u);  // let the row load land before the CTA exits
+    }
+    return;
+  }
+
+  if (counts_cta) {
+    // 2c. the counts and offsets of the whole batch
+    for (int tt = tid; tt < T; tt += kTokThreads) {
+      unsigned long long rm = 0ull;  // ranks of token tt's kept slots (R <= 64)
+      for (int j = 0; j < k; ++j) {
+        const int e = ids[tt * k + j];
+        if (e >= 0) rm |= 1ull << ((static_cast<unsigned long long>(e) * a.g_magic) >> 32);
+      }
+      while (rm != 0ull) {
+        atomicAdd(&cnt_r[__ffsll(static_cast<long long>(rm)) - 1], 1);
+        rm &= rm - 1ull;
+      }
+    }
+    token_cta_exclusive_scan(cnt, off, E, warp_tot);
+    __syncthreads();
+    const int n_eff = off[E];
+    for (int q = tid; q < E; q += kTokThreads) {
+      a.cnt_e[q] = cnt[q];
+      a.off_e[q] = off[q];
+    }
+    if (tid == 0) a.off_e[E] = n_eff;
+    if (warp == kTokWarps - 1) {
+      int carry = 0;
+      for (int b = 0; b < R; b += 32) {
+        const int r = b + lane;
+        const int c = r < R ? cnt_r[r] : 0;
+        const int incl = warp_incl_scan(c);
+        if (r < R) {
+          a.cnt_r[r] = c;
+          a.off_r[r] = carry + incl - c;
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) a.off_r[R] = carry;
+    }
+    for (int r = n_eff + tid; r < N; r += kTokThreads) a.recv_src[r] = -1;  // rows nobody fills
+    return;
+  }
+
+  // 2d. receive rows of this token's k slots: count the smaller keys
+  const int f0 = t * k;
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    int ej[8], c[8];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      ej[jj] = j0 + jj < k ? ids[f0 + j0 + jj] : -1;
+      c[jj] = 0;
+    }
+    for (int q = tid; q < N; q += kTokThreads) {
+      const int e = ids[q];
+      if (e < 0) continue;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj)
+        c[jj] += e < ej[jj] || (e == ej[jj] && q < f0 + j0 + jj);
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int sum = __reduce_add_sync(0xffffffffu, c[jj]);
+      if (lane == 0 && sum != 0 && j0 + jj < k) atomicAdd(&rank_sm[j0 + jj], sum);
+    }
+  }
+  __syncthreads();
+
+  // 3. layout entries of the token; lane j < k of warp 0 stores receive row j
+  if (warp == 1) {
+    for (int r = lane; r < R; r += 32) {
+      int in = 0;
+      for (int j = 0; j < k; ++j)
+        in |= static_cast<unsigned>(ids[f0 + j] - r * G) < static_cast<unsigned>(G);
+      a.in_rank[static_cast<long>(t) * R + r] = static_cast<uint8_t>(in);
+    }
+  }
+  if (warp == 0 && lane < k) {
+    const int row = ids[f0 + lane] >= 0 ? rank_sm[lane] : -1;
+    a.slot_pos[f0 + lane] = row;
+    if (row >= 0) {
+      a.recv_src[row] = t;
+      if (kFp8) {
+        const int nb = H >> 7;
+        bulk_store(a.recv + static_cast<long>(row) * H, out_q, H);
+        bulk_store(a.recv_scale + static_cast<long>(row) * nb, out_s, 4 * nb);
+      } else {
+        bulk_store(a.recv + static_cast<long>(row) * 2 * H, in_buf, 2 * H);
+      }
+      bulk_commit();
+      bulk_wait<0>();
+    }
+  }
+}
+
+template <typename IdT, bool kFp8>
+cudaError_t launch_token_kernel(const FusedArgs &a, cudaStream_t s) {
+  auto kern = layout_dispatch_token_kernel<IdT, kFp8>;
+  const int smem = token_smem_map(a.T, a.k, a.E, a.R, a.H, kFp8).total;
+  const cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(kern, dim3(a.T + 1), dim3(kTokThreads), smem, s, 1, a);
+}
+
+// CTAs of the token kernel that fit on `num_sms` SMs at once (0 = all).
+template <typename IdT, bool kFp8>
+long token_kernel_capacity(const FusedArgs &a, int num_sms) {
+  const int smem = token_smem_map(a.T, a.k, a.E, a.R, a.H, kFp8).total;
+  return persistent_grid(reinterpret_cast<const void *>(layout_dispatch_token_kernel<IdT, kFp8>),
+                         kTokThreads, smem, 1L << 40, num_sms);
+}
+
 template <typename IdT, bool kFp8>
 cudaError_t launch_fused(const FusedArgs &base, int num_sms, cudaStream_t s) {
+  if (base.T + 1 <= token_kernel_capacity<IdT, kFp8>(base, num_sms))
+    return launch_token_kernel<IdT, kFp8>(base, s);
   auto kern = layout_dispatch_kernel<IdT, kFp8>;
   // shared memory sized for ceil(T / SMs) tokens per CTA, which bounds the
   // tokens of a CTA below (at least one CTA per SM fits)

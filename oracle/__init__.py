@@ -64,6 +64,14 @@ def lib():
             _u16p, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             _i32p, _f32p, _u16p]
         L.ep_oracle_combine.restype = ctypes.c_int
+        L.ep_oracle_layout_aligned.argtypes = [
+            _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            _i32p, _i32p, _i32p]
+        L.ep_oracle_layout_aligned.restype = ctypes.c_int
+        L.ep_oracle_combine_fp8.argtypes = [
+            _u8p, _f32p, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            _i32p, _f32p, _u16p]
+        L.ep_oracle_combine_fp8.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -73,6 +81,8 @@ def _np(a, dtype) -> np.ndarray:
     if isinstance(a, torch.Tensor):
         if a.dtype == torch.bfloat16:
             a = a.view(torch.int16)
+        elif a.dtype == torch.float8_e4m3fn:
+            a = a.view(torch.uint8)
         a = a.detach().cpu().contiguous().numpy()
     a = np.ascontiguousarray(a)
     if a.dtype != dtype:
@@ -228,4 +238,49 @@ def combine(y, slot_pos, w) -> np.ndarray:
                                  _ptr(out, _u16p))
     if st:
         raise ValueError("oracle combine: invalid arguments")
+    return out
+
+
+# ------------------------------------------------------- aligned layout
+
+def padded_rows(T: int, k: int, E: int, align: int) -> int:
+    """Receive rows an aligned layout may use: T*k + E*(align-1)."""
+    return T * k + E * (align - 1)
+
+
+def layout_aligned(idx, E: int, align: int) -> Dict[str, np.ndarray]:
+    """Receive rows with every expert segment starting on a multiple of
+    ``align``: off_pad [E+1], slot_pos [T,k], recv_src [T*k + E*(align-1)]
+    (-1 for padding and unused rows) and the status."""
+    ix = _np(idx, np.int64)
+    T, k = ix.shape
+    out = {"off_pad": np.zeros(E + 1, np.int32),
+           "slot_pos": np.zeros((T, k), np.int32),
+           "recv_src": np.zeros(padded_rows(T, k, E, align), np.int32)}
+    st = lib().ep_oracle_layout_aligned(
+        _ptr(ix, _i64p), T, k, E, align, _ptr(out["off_pad"], _i32p),
+        _ptr(out["slot_pos"], _i32p), _ptr(out["recv_src"], _i32p))
+    if st == ORACLE_ERR_INVALID_ARG:
+        raise ValueError("oracle layout_aligned: invalid arguments")
+    out["status"] = st
+    return out
+
+
+# ---------------------------------------------------------- FP8 combine
+
+def combine_fp8(yq, ys, slot_pos, w) -> np.ndarray:
+    """out[t] = bf16(fma chain over slots of w[t, j] * (e4m3(yq) * ys)), as
+    uint16 bf16 bits [T, H]; w=None means every weight is 1."""
+    q = _np(yq, np.uint8)
+    sc = _np(ys, np.float32)
+    sp = _np(slot_pos, np.int32)
+    wf = np.ones(sp.shape, np.float32) if w is None else _np(w, np.float32)
+    n_rows, H = q.shape
+    T, k = sp.shape
+    assert sc.shape == (n_rows, H // 128)
+    out = np.zeros((T, H), np.uint16)
+    st = lib().ep_oracle_combine_fp8(_ptr(q, _u8p), _ptr(sc, _f32p), n_rows, T, H, k,
+                                     _ptr(sp, _i32p), _ptr(wf, _f32p), _ptr(out, _u16p))
+    if st:
+        raise ValueError("oracle combine_fp8: invalid arguments")
     return out

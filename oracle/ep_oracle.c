@@ -34,6 +34,18 @@
  *   combine  out[t,:] = bf16_rne( fma chain over j = 0..k-1 in slot order of
  *                       w[t,j] * y[slot_pos[t,j], :], starting from 0.0f )
  *
+ *   aligned layout (receive segments padded for a grouped GEMM whose row
+ *            tiles are `align` rows: each expert's segment starts on a
+ *            multiple of align)
+ *            off_pad      = exclusive prefix sum of ceil(cnt_e / align) * align
+ *            slot_pos[t,j]= off_pad[e] + the same stable rank as above
+ *            recv_src[r]  = token of row r, -1 for padding rows and past
+ *                           off_pad[E], over T*k + E*(align-1) rows
+ *   FP8 combine (expert outputs in the FP8 form of dispatch: e4m3 codes and
+ *            one fp32 scale per row and 128-channel block)
+ *            v = fp32(e4m3 value * scale), rounded to nearest
+ *            out[t,:] = bf16_rne( fma chain over j of w[t,j] * v )
+ *
  *   rank layout (the rank-deduplicated form of dispatch: one row per
  *            (token, rank) pair, DeepEP's per-peer sends)
  *            rank_row[t,r] = off_r[r] + #{t' < t : in_rank[t',r]} if
@@ -337,6 +349,95 @@ int ep_oracle_combine(const uint16_t *y, long n_rows, int T, int H, int k,
             for (int c = 0; c < H; ++c)
                 acc[c] = fmaf(wj, ep_oracle_bf16_to_f32(y[(long)row * H + c]),
                               acc[c]);
+        }
+        for (int c = 0; c < H; ++c)
+            out[(long)t * H + c] = ep_oracle_f32_to_bf16(acc[c]);
+    }
+    free(acc);
+    return EP_ORACLE_OK;
+}
+
+/* ------------------------------------------------------- aligned layout */
+
+/* Receive rows of the aligned layout: every expert's segment starts on a
+ * multiple of `align` rows (its used rows first, in the stable token-major
+ * order of ep_oracle_layout, then padding).  recv_src has n_cap =
+ * T*k + E*(align-1) entries.  Ids outside [0, E) are dropped (-1). */
+int ep_oracle_layout_aligned(const int64_t *idx, int T, int k, int E, int align,
+                             int32_t *off_pad, int32_t *slot_pos,
+                             int32_t *recv_src) {
+    if (T < 0 || k <= 0 || E <= 0 || align <= 0)
+        return EP_ORACLE_ERR_INVALID_ARG;
+    const long N = (long)T * k;
+    const long n_cap = N + (long)E * (align - 1);
+    int32_t *cnt = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+    int32_t *next = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    if (!cnt || !next) {
+        free(cnt);
+        free(next);
+        return EP_ORACLE_ERR_INVALID_ARG;
+    }
+    int status = EP_ORACLE_OK;
+    for (long i = 0; i < N; ++i) {
+        const int64_t e = idx[i];
+        if (e >= 0 && e < E)
+            cnt[e] += 1;
+        else if (e != -1)
+            status = EP_ORACLE_ERR_INDEX;
+    }
+    off_pad[0] = 0;
+    for (int e = 0; e < E; ++e) {
+        const int32_t padded = (cnt[e] + align - 1) / align * align;
+        off_pad[e + 1] = off_pad[e] + padded;
+        next[e] = off_pad[e];
+    }
+    for (long r = 0; r < n_cap; ++r)
+        recv_src[r] = -1;
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            const long i = (long)t * k + j;
+            const int64_t e = idx[i];
+            if (e < 0 || e >= E) {
+                slot_pos[i] = -1;
+                continue;
+            }
+            const int32_t row = next[e]++;
+            slot_pos[i] = row;
+            recv_src[row] = t;
+        }
+    }
+    free(cnt);
+    free(next);
+    return status;
+}
+
+/* ---------------------------------------------------------- FP8 combine */
+
+/* Gate-weighted combine of expert outputs given as e4m3 codes yq [n_rows, H]
+ * and fp32 scales ys [n_rows, H/128]: each value is decoded and multiplied
+ * by its block's scale in fp32, then folded into the fp32 fma chain. */
+int ep_oracle_combine_fp8(const uint8_t *yq, const float *ys, long n_rows, int T,
+                          int H, int k, const int32_t *slot_pos, const float *w,
+                          uint16_t *out) {
+    if (T < 0 || H <= 0 || k <= 0 || H % 128 != 0)
+        return EP_ORACLE_ERR_INVALID_ARG;
+    const int nb = H / 128;
+    float *acc = (float *)malloc(sizeof(float) * (size_t)H);
+    if (!acc)
+        return EP_ORACLE_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t) {
+        for (int c = 0; c < H; ++c)
+            acc[c] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int32_t row = slot_pos[(long)t * k + j];
+            if (row < 0 || row >= n_rows)
+                continue;
+            const float wj = w[(long)t * k + j];
+            for (int c = 0; c < H; ++c) {
+                const float v = ep_oracle_e4m3_to_f32(yq[(long)row * H + c]) *
+                                ys[(long)row * nb + c / 128];
+                acc[c] = fmaf(wj, v, acc[c]);
+            }
         }
         for (int c = 0; c < H; ++c)
             out[(long)t * H + c] = ep_oracle_f32_to_bf16(acc[c]);

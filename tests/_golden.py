@@ -50,3 +50,16 @@ def combine_case():
         key, vals = line.split(":", 1)
         d[key.strip()] = [float(v) for v in vals.split()]
     return d
+
+
+def layout_aligned_cases():
+    cases, cur = [], None
+    for line in _lines("layout_aligned_hand.txt"):
+        if line.startswith("case"):
+            T, k, E, align = map(int, line.split()[1:])
+            cur = dict(T=T, k=k, E=E, align=align)
+            cases.append(cur)
+        else:
+            key, vals = line.split(":", 1)
+            cur[key.strip()] = [int(v) for v in vals.split()]
+    return cases

@@ -155,6 +155,20 @@ def test_bad_ids_reported_and_dropped():
     assert _check(idx, b.x, cfg.E, cfg.R, True) == 1
 
 
+@pytest.mark.parametrize("num_sms", [0, 1, 2])
+@pytest.mark.parametrize("fp8", [False, True])
+def test_both_fused_kernels_on_the_decode_shape(num_sms, fp8):
+    # all SMs: one token per CTA (T + 1 CTAs fit at once); one or two SMs:
+    # the token-range kernel, each CTA walking many tokens through its
+    # two-stage row pipeline -- with dropped, duplicated and bad ids
+    cfg, b = _batch("decode", 22, drop_frac=0.05, dup_frac=0.1)
+    idx = b.idx.clone()
+    idx[5, 2] = 999
+    host, _, _ = _run(idx, b.x, cfg.E, cfg.R, fp8, num_sms=num_sms)
+    assert host["status"] == ep.EP_ERR_INDEX
+    assert _check(idx, b.x, cfg.E, cfg.R, fp8, num_sms=num_sms) == 1
+
+
 @pytest.mark.parametrize("H,fused", [(8, True), (136, True), (7176, True), (16384, True),
                                      (16392, False)])
 def test_bf16_hidden_sizes(H, fused):
