@@ -351,6 +351,8 @@ def bench_ours(args, world, rank, device):
         result["decode"] = bench_decode(ep, device, world)
     if not args.skip_dedup:
         result["rank_dedup"] = bench_rank_dedup(ep, st, cfg, device, world)
+    if not args.skip_variants:
+        result["combine_variants"] = bench_combine_variants(ep, st, cfg, device, world)
     if not args.skip_overlap:
         result["sm_budget_overlap"] = bench_overlap(ep, st, cfg, device, world)
     if not args.skip_e2e:
@@ -368,6 +370,7 @@ KERNEL_SOURCES = {
     "dispatch_fp8": ("dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
     "combine": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),
     "layout_dispatch_fp8": ("layout_dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
+    "combine_fp8": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),
 }
 
 
@@ -447,6 +450,60 @@ def bench_rank_dedup(ep, st, cfg, device, world, iters=20):
                             world, device)
         res[name] = {"us": round(us, 2), "bytes": nbytes,
                      "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)}
+    return res
+
+
+def bench_combine_variants(ep, st, cfg, device, world, iters=20, align=128):
+    """The combine variants on the prefill batch, each kernel timed alone
+    (flushed L2): the aligned layout for a grouped GEMM with `align`-row
+    tiles, the FP8 dispatch into that padded buffer, and the combine of FP8
+    expert outputs (the FP8 receive rows themselves: identity experts)."""
+    T, H, k, E = cfg.T, cfg.H, cfg.k, cfg.E
+    stream = torch.cuda.Stream(device)
+    flush = L2Flush(device)
+    with torch.cuda.stream(stream):
+        st.run(stream)
+        pl = ep.ep_pad_layout(st.layout, align, stream=stream)
+    stream.synchronize()
+    cap = ep.ep_aligned_rows(T, k, E, align)
+    q = torch.zeros((cap, H), dtype=torch.float8_e4m3fn, device=device)
+    sc = torch.zeros((cap, H // 128), dtype=torch.float32, device=device)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    N = T * k
+    calls = {
+        "pad_layout": (lambda: ep.ep_pad_layout(st.layout, align, out=pl, stream=stream),
+                       E * 4 + N * 4 + (E + 1) * 4 + N * 4 + cap * 4),
+        "dispatch_fp8_padded": (lambda: ep.ep_dispatch(st.x, pl.slot_pos, fp8=True, recv=q,
+                                                       recv_scale=sc, d_err=st.d_err,
+                                                       stream=stream),
+                                T * H * 2 + N * (H + H // 32)),
+        "combine_fp8": (lambda: ep.ep_combine_fp8(q, sc, pl.slot_pos, st.w, out=out,
+                                                  d_err=st.d_err, stream=stream),
+                        N * (H + H // 32) + T * H * 2),
+    }
+    res = {"align": align, "rows": cap, "rows_in_use": None}
+    for name, (fn, nbytes) in calls.items():
+        evs = []
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                flush()
+                fn()
+            for _ in range(iters):
+                flush()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                evs.append((a, b))
+        stream.synchronize()
+        us = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3,
+                            world, device)
+        res[name] = {"us": round(us, 2), "bytes": nbytes,
+                     "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)}
+    res["rows_in_use"] = int(pl.off_pad[-1].item())
+    if ep.ep_read_error(st.d_err, stream) != 0:
+        raise RuntimeError("the device reported an error in the combine variants")
     return res
 
 
@@ -780,6 +837,8 @@ def profile_kernel(args, device):
         "layout_dispatch_fp8": lambda: ep.ep_layout_dispatch(
             st.idx, c.E, c.R, st.x, True, out=st.layout, recv=st.recv_q,
             recv_scale=st.recv_s, ws=st.ws, d_err=st.d_err, stream=stream),
+        "combine_fp8": lambda: ep.ep_combine_fp8(st.recv_q, st.recv_s, st.layout.slot_pos, st.w,
+                                                 out=st.out, d_err=st.d_err, stream=stream),
     }
     call = calls[args.profile]
     with torch.cuda.stream(stream):
@@ -815,10 +874,11 @@ def main():
     p.add_argument("--skip-cpu", action="store_true")
     p.add_argument("--skip-dedup", action="store_true")
     p.add_argument("--skip-overlap", action="store_true")
+    p.add_argument("--skip-variants", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--reference-tokens", type=int, default=256)
     p.add_argument("--profile", choices=("layout", "dispatch_bf16", "dispatch_fp8", "combine",
-                                         "layout_dispatch_fp8"),
+                                         "layout_dispatch_fp8", "combine_fp8"),
                    help="run only this kernel (for profiler captures)")
     p.add_argument("--workload", choices=tuple(workloads.CONFIGS), default="prefill",
                    help="workload of --profile")

@@ -24,6 +24,7 @@ __all__ = ["EPError", "EPLibraryError", "Layout", "RankLayout", "ep_get_layout",
            "ep_get_rank_layout", "ep_rank_layout_workspace_bytes",
            "ep_get_layout_noalloc", "EP_NOALLOC_SCRATCH_BYTES",
            "ep_dispatch", "ep_combine", "ep_read_error", "ep_layout_dispatch",
+           "ep_combine_fp8", "ep_aligned_rows", "ep_pad_layout", "PaddedLayout",
            "ep_layout_workspace_bytes", "ep_kernel_launches", "lib",
            "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_UNSUPPORTED", "EP_ERR_CUDA",
            "EP_ERR_INDEX", "EP_ERR_TIMEOUT", "LIB_PATH"]
@@ -62,8 +63,11 @@ _SIGNATURES = {
     "ep_layout_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "ep_get_layout": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                        _vp, _vp, _sz, _vp, _vp], _i),
-    "ep_dispatch": ([_vp, _i, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp], _i),
-    "ep_combine": ([_vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp], _i),
+    "ep_dispatch": ([_vp, _i, _i, _i, _vp, _i, _vp, _vp, _i, _i, _vp, _vp], _i),
+    "ep_combine": ([_vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp], _i),
+    "ep_combine_fp8": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp], _i),
+    "ep_aligned_rows": ([_i, _i, _i, _i], _sz),
+    "ep_pad_layout": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
     "ep_read_error": ([_vp, _vp], _i),
     "ep_get_layout_noalloc": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                _vp, _vp, _vp, _vp], _i),
@@ -234,7 +238,8 @@ def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
                 stream=None):
     """Rows of ``x`` [T, H] bf16 to their receive rows.  Returns ``recv``
     [T*k, H] (bf16), or ``(recv_q [T*k, H] float8_e4m3fn, recv_scale
-    [T*k, H/128] fp32)`` when ``fp8``."""
+    [T*k, H/128] fp32)`` when ``fp8``.  A given ``recv`` may have more rows
+    (an aligned layout's ep_aligned_rows); slot rows past it are skipped."""
     _need_cuda("x", x)
     _need_cuda("slot_pos", slot_pos)
     if x.dtype != torch.bfloat16 or slot_pos.dtype != torch.int32:
@@ -245,11 +250,15 @@ def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
         recv = torch.empty((T * k, H), device=x.device,
                            dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16)
     if fp8 and recv_scale is None:
-        recv_scale = torch.empty((T * k, H // 128), device=x.device,
+        recv_scale = torch.empty((recv.shape[0], H // 128), device=x.device,
                                  dtype=torch.float32)
+    if fp8 and recv_scale.shape[0] < recv.shape[0]:
+        raise ValueError("recv_scale needs a row per receive row")
+    if recv.shape[0] == 0 and T * k > 0:
+        raise ValueError("recv has no rows")   # 0 would mean T*k rows to the library
     _check(lib().ep_dispatch(_ptr(x), T, H, k, _ptr(slot_pos), int(bool(fp8)),
                              _ptr(recv), _ptr(recv_scale) if fp8 else None,
-                             num_sms, _ptr(d_err), _stream(stream)))
+                             recv.shape[0], num_sms, _ptr(d_err), _stream(stream)))
     return (recv, recv_scale) if fp8 else recv
 
 
@@ -305,12 +314,66 @@ def ep_combine(y: torch.Tensor, slot_pos: torch.Tensor, w: Optional[torch.Tensor
         raise ValueError("y must be bf16 and w fp32")
     T, k = slot_pos.shape
     H = y.shape[1]
-    if y.shape[0] < T * k:
-        raise ValueError(f"y needs at least T*k={T * k} rows")
     if out is None:
         out = torch.empty((T, H), device=y.device, dtype=torch.bfloat16)
-    _check(lib().ep_combine(_ptr(y), T, H, k, _ptr(slot_pos), _ptr(w),
+    if y.shape[0] == 0 and T > 0:
+        raise ValueError("y has no rows")   # 0 would mean T*k rows to the library
+    _check(lib().ep_combine(_ptr(y), y.shape[0], T, H, k, _ptr(slot_pos), _ptr(w),
                             _ptr(out), num_sms, _ptr(d_err), _stream(stream)))
+    return out
+
+
+def ep_combine_fp8(y_q: torch.Tensor, y_scale: torch.Tensor, slot_pos: torch.Tensor,
+                   w: Optional[torch.Tensor], *, out: Optional[torch.Tensor] = None,
+                   num_sms: int = 0, d_err: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Gate-weighted combine of FP8 expert outputs (``y_q`` [rows, H]
+    float8_e4m3fn codes, ``y_scale`` [rows, H/128] fp32) into ``out`` [T, H]
+    bf16: each value decoded and scaled in fp32, then the fp32 fma chain in
+    slot order."""
+    for name, t in (("y_q", y_q), ("y_scale", y_scale), ("slot_pos", slot_pos)):
+        _need_cuda(name, t)
+    if w is not None:
+        _need_cuda("w", w)
+    if y_q.dtype != torch.float8_e4m3fn or y_scale.dtype != torch.float32:
+        raise ValueError("y_q must be float8_e4m3fn and y_scale fp32")
+    T, k = slot_pos.shape
+    rows, H = y_q.shape
+    if (rows == 0 and T > 0) or y_scale.shape != (rows, H // 128):
+        raise ValueError("y_scale must be [rows, H/128] and y_q hold rows")
+    if out is None:
+        out = torch.empty((T, H), device=y_q.device, dtype=torch.bfloat16)
+    _check(lib().ep_combine_fp8(_ptr(y_q), _ptr(y_scale), rows, T, H, k, _ptr(slot_pos),
+                                _ptr(w), _ptr(out), num_sms, _ptr(d_err), _stream(stream)))
+    return out
+
+
+class PaddedLayout(NamedTuple):
+    off_pad: torch.Tensor       # [E+1] int32
+    slot_pos: torch.Tensor      # [T, k] int32, rows of the aligned buffer
+    recv_src: torch.Tensor      # [ep_aligned_rows(T, k, E, align)] int32
+
+
+def ep_aligned_rows(T: int, k: int, E: int, align: int) -> int:
+    return int(lib().ep_aligned_rows(T, k, E, align))
+
+
+def ep_pad_layout(layout: Layout, align: int, *, out: Optional[PaddedLayout] = None,
+                  stream=None) -> PaddedLayout:
+    """Expert segments of ``layout`` (from ep_get_layout) moved to start on
+    multiples of ``align`` rows, for a grouped GEMM with row tiles of that
+    size.  Dispatch into and combine from a buffer of
+    ``ep_aligned_rows(T, k, E, align)`` rows with the returned slot_pos."""
+    T, k = layout.slot_pos.shape
+    E = layout.cnt_e.shape[0]
+    dev = layout.slot_pos.device
+    if out is None:
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = PaddedLayout(torch.empty(E + 1, **i32), torch.empty((T, k), **i32),
+                           torch.empty(max(1, ep_aligned_rows(T, k, E, align)), **i32))
+    _check(lib().ep_pad_layout(_ptr(layout.cnt_e), _ptr(layout.slot_pos), T, k, E, align,
+                               _ptr(out.off_pad), _ptr(out.slot_pos), _ptr(out.recv_src),
+                               _stream(stream)))
     return out
 
 

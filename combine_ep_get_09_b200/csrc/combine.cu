@@ -17,6 +17,8 @@
 //  * combine_reg_kernel (any k <= 32): a warp per item with 128-bit loads
 //    of 8 slot rows at a time into registers.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "bulk.cuh"
 #include "ep_internal.cuh"
@@ -182,13 +184,215 @@ __global__ void __launch_bounds__(kRegThreads, 2)
   }
 }
 
+// ------------------------------------------------------------ FP8 combine
+//
+// Expert outputs in the FP8 form of dispatch: e4m3 codes y_q [rows, H] and
+// one fp32 scale per row and 128-channel block.  Each value is decoded
+// (exact), multiplied by its scale in fp32 (round to nearest) and folded
+// into the same fp32 fma chain in slot order as the bf16 combine.
+
+// 16 e4m3 codes -> 16 floats (exact: every e4m3 value is a half).
+__device__ __forceinline__ void decode_e4m3x16(uint4 v, float *f) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __nv_fp8x2_storage_t pair =
+          static_cast<__nv_fp8x2_storage_t>((in[i] >> (16 * h)) & 0xffffu);
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      const float2 ff = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+      f[4 * i + 2 * h] = ff.x;
+      f[4 * i + 2 * h + 1] = ff.y;
+    }
+  }
+}
+
+__device__ __forceinline__ void fma_e4m3x16(float *acc, float w, uint4 q, float scale) {
+  float f[16];
+  decode_e4m3x16(q, f);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = __fmaf_rn(w, __fmul_rn(f[e], scale), acc[e]);
+}
+
+__device__ __forceinline__ void store_bf16x16(uint4 *dst, const float *acc) {
+  st_stream_v4(dst, to_bf16x8(acc));
+  st_stream_v4(dst + 1, to_bf16x8(acc + 8));
+}
+
+constexpr int kQChunkVec = 256;  // 16-byte code vectors (4096 channels) per item
+constexpr int kQStageBytes = kBulkMaxK * (kQChunkVec * 16 + kQChunkVec / 8 * 4);
+constexpr int kQBulkSmem = kStages * kQStageBytes;
+
+// Bulk-copy pipeline as combine_bulk_kernel (k <= 8; H % 512 == 0 so every
+// chunk's codes and scales are whole 16-byte units): item = (token, chunk
+// of 4096 channels); lane j < k of warp 0 gathers slot row j's codes and
+// its 32 block scales; thread v folds 16 channels of every row.
+__global__ void __launch_bounds__(kQChunkVec)
+    combine_fp8_bulk_kernel(const uint4 *__restrict__ y_q, const float *__restrict__ y_scale,
+                            int T, int H, int k, const int32_t *__restrict__ slot_pos,
+                            const float *__restrict__ w, uint4 *__restrict__ out, long n_rows,
+                            int32_t *d_err) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ int stage_row[kStages][kBulkMaxK];
+  __shared__ float stage_w[kStages][kBulkMaxK];
+
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int Hq = H >> 4;  // code vectors per row
+  const int nb = H >> 7;  // scales per row
+  const int nchunks = (Hq + kQChunkVec - 1) / kQChunkVec;
+  const long items = static_cast<long>(T) * nchunks;
+  const long first = items * blockIdx.x / gridDim.x;
+  const long n_mine = items * (blockIdx.x + 1) / gridDim.x - first;
+  auto codes = [&](int s, int j) {
+    return reinterpret_cast<uint4 *>(smem_raw + s * kQStageBytes) + j * kQChunkVec;
+  };
+  auto scales = [&](int s, int j) {
+    return reinterpret_cast<float *>(smem_raw + s * kQStageBytes +
+                                     kBulkMaxK * kQChunkVec * 16) +
+           j * (kQChunkVec / 8);
+  };
+
+  pdl_trigger();
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], kWarp);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  pdl_wait();
+
+  auto issue = [&](long i) {  // warp 0, as in combine_bulk_kernel
+    const long it = first + i;
+    const int s = static_cast<int>(i % kStages);
+    const int t = static_cast<int>(it / nchunks);
+    const int v0 = static_cast<int>(it % nchunks) * kQChunkVec;
+    const int nv = min(kQChunkVec, Hq - v0);
+    int r = -1;
+    if (lane < k) {
+      r = __ldg(slot_pos + static_cast<long>(t) * k + lane);
+      const float wj = w != nullptr ? __ldg(w + static_cast<long>(t) * k + lane) : 1.0f;
+      if (r < 0 || r >= n_rows) r = -1;
+      stage_row[s][lane] = r;
+      stage_w[s][lane] = wj;
+    } else if (lane < kBulkMaxK) {
+      stage_row[s][lane] = -1;
+    }
+    const unsigned code_bytes = static_cast<unsigned>(nv) * 16u;
+    const unsigned scale_bytes = static_cast<unsigned>(nv / 8) * 4u;
+    mbar_arrive_expect_tx(&full[s], r >= 0 ? code_bytes + scale_bytes : 0u);
+    if (r >= 0) {
+      bulk_load(codes(s, lane), y_q + static_cast<long>(r) * Hq + v0, code_bytes, &full[s]);
+      bulk_load(scales(s, lane), y_scale + static_cast<long>(r) * nb + v0 / 8, scale_bytes,
+                &full[s]);
+    }
+  };
+
+  if (tid < kWarp)
+    for (long i = 0; i < min(static_cast<long>(kStages), n_mine); ++i) issue(i);
+
+  long i = 0;
+  bool timed_out = false;
+  for (; i < n_mine; ++i) {
+    const int s = static_cast<int>(i % kStages);
+    const long it = first + i;
+    const int t = static_cast<int>(it / nchunks);
+    const int v0 = static_cast<int>(it % nchunks) * kQChunkVec;
+    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1));
+    if (__syncthreads_or(!ok)) {
+      timed_out = true;
+      break;
+    }
+    if (tid < Hq - v0) {
+      float acc[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < kBulkMaxK; ++j)
+        if (stage_row[s][j] >= 0)
+          fma_e4m3x16(acc, stage_w[s][j], codes(s, j)[tid], scales(s, j)[tid >> 3]);
+      store_bf16x16(out + (static_cast<long>(t) * Hq + v0 + tid) * 2, acc);
+    }
+    __syncthreads();  // stage s fully read
+    if (tid < kWarp && i + kStages < n_mine) issue(i + kStages);
+  }
+  if (timed_out && tid == 0) {
+    if (d_err != nullptr) atomicExch(reinterpret_cast<int *>(d_err), EP_ERR_TIMEOUT);
+    for (long q = i; q < min(n_mine, i + kStages); ++q)
+      mbar_wait_bounded(&full[q % kStages], static_cast<unsigned>((q / kStages) & 1));
+  }
+}
+
+// Any k <= 32 and H % 128 == 0: a warp per (token, 512 channels), the
+// lane's 16 codes and their scale read directly.
+__global__ void __launch_bounds__(kRegThreads, 2)
+    combine_fp8_reg_kernel(const uint4 *__restrict__ y_q, const float *__restrict__ y_scale,
+                           int T, int H, int k, const int32_t *__restrict__ slot_pos,
+                           const float *__restrict__ w, uint4 *__restrict__ out,
+                           long n_rows) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int Hq = H >> 4, nb = H >> 7;
+  const int nchunks = (Hq + 31) / 32;
+  const long items = static_cast<long>(T) * nchunks;
+  const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
+  for (long it = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       it < items; it += nwarps) {
+    const int t = static_cast<int>(it / nchunks);
+    const int v = static_cast<int>(it - static_cast<long>(t) * nchunks) * 32 + lane;
+    const long tk = static_cast<long>(t) * k;
+    const int sp = lane < k ? __ldg(slot_pos + tk + lane) : -1;
+    const float wt = lane < k ? (w != nullptr ? __ldg(w + tk + lane) : 1.0f) : 0.0f;
+    float acc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int row = __shfl_sync(0xffffffffu, sp, j);
+      const float wj = __shfl_sync(0xffffffffu, wt, j);
+      if (row < 0 || row >= n_rows || v >= Hq) continue;
+      fma_e4m3x16(acc, wj, ld_stream_v4(y_q + static_cast<long>(row) * Hq + v),
+                  __ldg(y_scale + static_cast<long>(row) * nb + (v >> 3)));
+    }
+    if (v < Hq) store_bf16x16(out + (static_cast<long>(t) * Hq + v) * 2, acc);
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_combine(const void *y, int T, int H, int k, const int32_t *slot_pos,
-                           const float *w, void *out, int num_sms, int32_t *d_err,
-                           cudaStream_t s, int *launches) {
+cudaError_t launch_combine_fp8(const void *y_q, const float *y_scale, long n_rows, int T,
+                               int H, int k, const int32_t *slot_pos, const float *w,
+                               void *out, int num_sms, int32_t *d_err, cudaStream_t s,
+                               int *launches) {
+  const int Hq = H / 16;
+  if (k <= kBulkMaxK && H % 512 == 0 && reinterpret_cast<uintptr_t>(y_scale) % 16 == 0) {
+    const long items = static_cast<long>(T) * ((Hq + kQChunkVec - 1) / kQChunkVec);
+    if (items == 0) return cudaSuccess;
+    const cudaError_t err = raise_dynamic_smem(
+        reinterpret_cast<const void *>(combine_fp8_bulk_kernel), kQBulkSmem);
+    if (err != cudaSuccess) return err;
+    const long grid = persistent_grid(reinterpret_cast<const void *>(combine_fp8_bulk_kernel),
+                                      kQChunkVec, kQBulkSmem, items * (kQChunkVec / kWarp),
+                                      num_sms);
+    ++*launches;
+    return launch_pdl(combine_fp8_bulk_kernel, dim3(grid), dim3(kQChunkVec), kQBulkSmem, s, 1,
+                      static_cast<const uint4 *>(y_q), y_scale, T, H, k, slot_pos, w,
+                      static_cast<uint4 *>(out), n_rows, d_err);
+  }
+  const long items = static_cast<long>(T) * ((Hq + 31) / 32);
+  if (items == 0) return cudaSuccess;
+  const long grid = persistent_grid(reinterpret_cast<const void *>(combine_fp8_reg_kernel),
+                                    kRegThreads, 0, items, num_sms);
+  ++*launches;
+  return launch_pdl(combine_fp8_reg_kernel, dim3(grid), dim3(kRegThreads), 0, s, 1,
+                    static_cast<const uint4 *>(y_q), y_scale, T, H, k, slot_pos, w,
+                    static_cast<uint4 *>(out), n_rows);
+}
+
+cudaError_t launch_combine(const void *y, long n_rows, int T, int H, int k,
+                           const int32_t *slot_pos, const float *w, void *out, int num_sms,
+                           int32_t *d_err, cudaStream_t s, int *launches) {
   const int Hv = H / 8;
-  const long n_rows = static_cast<long>(T) * k;
   if (k <= kBulkMaxK) {
     const long items = static_cast<long>(T) * ((Hv + kChunkVec - 1) / kChunkVec);
     if (items == 0) return cudaSuccess;

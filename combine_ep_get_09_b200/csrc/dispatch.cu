@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kThreads)
 }  // namespace
 
 cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
-                                 const int32_t *slot_pos, void *recv,
+                                 const int32_t *slot_pos, void *recv, long n_rows,
                                  int num_sms, int32_t * /*d_err*/, cudaStream_t s,
                                  int *launches) {
   const int Hv = H / 8;
@@ -224,7 +224,7 @@ cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
       persistent_grid(reinterpret_cast<const void *>(kern), kThreads, 0, items, num_sms);
   ++*launches;
   return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, s, 1, static_cast<const uint4 *>(x), T,
-                    Hv, k, slot_pos, static_cast<uint4 *>(recv), static_cast<long>(T) * k);
+                    Hv, k, slot_pos, static_cast<uint4 *>(recv), n_rows);
 }
 
 // Largest hidden size the bulk FP8 kernel stages in shared memory.
@@ -234,7 +234,7 @@ int fp8_bulk_smem(int H) { return kFp8BulkStages * 2 * H + H + H / 32; }
 
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
-                                float *recv_scale, int num_sms, int32_t *d_err,
+                                float *recv_scale, long n_rows, int num_sms, int32_t *d_err,
                                 cudaStream_t s, int *launches) {
   // bulk stores need 16-byte aligned scale rows: H % 512 == 0 and an
   // aligned recv_scale
@@ -252,8 +252,7 @@ cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
     ++*launches;
     return launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(kFp8BulkThreads), smem, s, 1,
                       static_cast<const uint4 *>(x), T, H, k, slot_pos,
-                      static_cast<uint8_t *>(recv_q), recv_scale, static_cast<long>(T) * k,
-                      d_err);
+                      static_cast<uint8_t *>(recv_q), recv_scale, n_rows, d_err);
   }
   const long nchunks = (H / 128 + 3) / 4;
   const long items = static_cast<long>(T) * nchunks;
@@ -263,7 +262,7 @@ cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
   ++*launches;
   return launch_pdl(dispatch_fp8_kernel, dim3(grid), dim3(kThreads), 0, s, 1,
                     static_cast<const uint4 *>(x), T, H, k, slot_pos,
-                    static_cast<uint2 *>(recv_q), recv_scale, static_cast<long>(T) * k);
+                    static_cast<uint2 *>(recv_q), recv_scale, n_rows);
 }
 
 }  // namespace ep

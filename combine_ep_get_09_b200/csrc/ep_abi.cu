@@ -130,7 +130,7 @@ cudaError_t raise_dynamic_smem(const void *kernel, int bytes) {
 
 extern "C" {
 
-int ep_abi_version(void) { return 3; }
+int ep_abi_version(void) { return 4; }
 
 const char *ep_last_error_string(void) { return g_err; }
 
@@ -265,12 +265,23 @@ ep_status_t ep_get_rank_layout(const uint8_t *in_rank, int T, int R, int32_t *cn
   return from_cuda(e, fn);
 }
 
+// Rows of a receive buffer: recv_rows, or T*k when it is 0.
+static ep_status_t receive_rows(const char *fn, int recv_rows, int T, int k, long *n_rows) {
+  if (recv_rows < 0) return fail(EP_ERR_INVALID_ARG, "%s: recv_rows=%d < 0", fn, recv_rows);
+  *n_rows = recv_rows > 0 ? recv_rows : static_cast<long>(T) * k;
+  return EP_OK;
+}
+
 ep_status_t ep_dispatch(const void *x, int T, int H, int k,
                         const int32_t *slot_pos, int fp8, void *recv,
-                        float *recv_scale, int num_sms, int32_t *d_err, void *stream) {
+                        float *recv_scale, int recv_rows, int num_sms, int32_t *d_err,
+                        void *stream) {
   static const char fn[] = "ep_dispatch";
   g_err[0] = '\0';
   ep_status_t st = check_rows(fn, T, H, k, num_sms);
+  if (st != EP_OK) return st;
+  long n_rows = 0;
+  st = receive_rows(fn, recv_rows, T, k, &n_rows);
   if (st != EP_OK) return st;
   if (fp8 && H % 128 != 0)
     return fail(EP_ERR_UNSUPPORTED, "%s: fp8 needs H %% 128 == 0 (H=%d)", fn, H);
@@ -284,8 +295,9 @@ ep_status_t ep_dispatch(const void *x, int T, int H, int k,
   int n = 0;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
-      fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale, num_sms, d_err, s, &n)
-          : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, num_sms, d_err, s, &n);
+      fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale, n_rows, num_sms,
+                                    d_err, s, &n)
+          : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, n_rows, num_sms, d_err, s, &n);
   g_launches += n;
   return from_cuda(e, fn);
 }
@@ -326,20 +338,24 @@ ep_status_t ep_layout_dispatch(const void *idx, int idx_is_int64, int T, int k, 
   } else {
     e = ep::launch_layout(a, s, &n);
     if (e == cudaSuccess)
-      e = fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale, num_sms, d_err,
-                                        s, &n)
-              : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, num_sms, d_err, s, &n);
+      e = fp8 ? ep::launch_dispatch_fp8(x, T, H, k, slot_pos, recv, recv_scale,
+                                        static_cast<long>(T) * k, num_sms, d_err, s, &n)
+              : ep::launch_dispatch_bf16(x, T, H, k, slot_pos, recv, static_cast<long>(T) * k,
+                                         num_sms, d_err, s, &n);
   }
   g_launches += n;
   return from_cuda(e, fn);
 }
 
-ep_status_t ep_combine(const void *y, int T, int H, int k,
+ep_status_t ep_combine(const void *y, int y_rows, int T, int H, int k,
                        const int32_t *slot_pos, const float *w, void *out,
                        int num_sms, int32_t *d_err, void *stream) {
   static const char fn[] = "ep_combine";
   g_err[0] = '\0';
   ep_status_t st = check_rows(fn, T, H, k, num_sms);
+  if (st != EP_OK) return st;
+  long n_rows = 0;
+  st = receive_rows(fn, y_rows, T, k, &n_rows);
   if (st != EP_OK) return st;
   if (T == 0) return EP_OK;
   EP_REQUIRE_PTR(fn, y, 16);
@@ -350,8 +366,70 @@ ep_status_t ep_combine(const void *y, int T, int H, int k,
   if (d_err != nullptr && !aligned(d_err, 4))
     return fail(EP_ERR_INVALID_ARG, "%s: d_err is not 4-byte aligned", fn);
   int n = 0;
-  const cudaError_t e = ep::launch_combine(y, T, H, k, slot_pos, w, out, num_sms, d_err,
+  const cudaError_t e = ep::launch_combine(y, n_rows, T, H, k, slot_pos, w, out, num_sms, d_err,
                                            static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
+  return from_cuda(e, fn);
+}
+
+ep_status_t ep_combine_fp8(const void *y_q, const float *y_scale, int y_rows, int T, int H,
+                           int k, const int32_t *slot_pos, const float *w, void *out,
+                           int num_sms, int32_t *d_err, void *stream) {
+  static const char fn[] = "ep_combine_fp8";
+  g_err[0] = '\0';
+  ep_status_t st = check_rows(fn, T, H, k, num_sms);
+  if (st != EP_OK) return st;
+  if (H % 128 != 0)
+    return fail(EP_ERR_UNSUPPORTED, "%s: H=%d is not a multiple of 128", fn, H);
+  long n_rows = 0;
+  st = receive_rows(fn, y_rows, T, k, &n_rows);
+  if (st != EP_OK) return st;
+  if (T == 0) return EP_OK;
+  EP_REQUIRE_PTR(fn, y_q, 16);
+  EP_REQUIRE_PTR(fn, y_scale, 4);
+  EP_REQUIRE_PTR(fn, slot_pos, 4);
+  if (w != nullptr && !aligned(w, 4))
+    return fail(EP_ERR_INVALID_ARG, "%s: w is not 4-byte aligned", fn);
+  EP_REQUIRE_PTR(fn, out, 16);
+  if (d_err != nullptr && !aligned(d_err, 4))
+    return fail(EP_ERR_INVALID_ARG, "%s: d_err is not 4-byte aligned", fn);
+  int n = 0;
+  const cudaError_t e =
+      ep::launch_combine_fp8(y_q, y_scale, n_rows, T, H, k, slot_pos, w, out, num_sms, d_err,
+                             static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
+  return from_cuda(e, fn);
+}
+
+size_t ep_aligned_rows(int T, int k, int E, int align) {
+  if (T < 0 || k < 1 || E < 1 || align < 1) return 0;
+  const long long rows = static_cast<long long>(T) * k + static_cast<long long>(E) * (align - 1);
+  return rows > 0x7fffffffLL ? 0 : static_cast<size_t>(rows);
+}
+
+ep_status_t ep_pad_layout(const int32_t *cnt_e, const int32_t *slot_pos, int T, int k, int E,
+                          int align, int32_t *off_pad, int32_t *slot_pos_pad,
+                          int32_t *recv_src_pad, void *stream) {
+  static const char fn[] = "ep_pad_layout";
+  g_err[0] = '\0';
+  if (T < 0) return fail(EP_ERR_INVALID_ARG, "%s: T=%d < 0", fn, T);
+  if (k < 1) return fail(EP_ERR_INVALID_ARG, "%s: k=%d < 1", fn, k);
+  if (E < 1) return fail(EP_ERR_INVALID_ARG, "%s: E=%d < 1", fn, E);
+  if (align < 1) return fail(EP_ERR_INVALID_ARG, "%s: align=%d < 1", fn, align);
+  if (E > EP_MAX_E) return fail(EP_ERR_UNSUPPORTED, "%s: E=%d > %d", fn, E, EP_MAX_E);
+  if (ep_aligned_rows(T, k, E, align) == 0 && T > 0)
+    return fail(EP_ERR_UNSUPPORTED, "%s: T*k + E*(align-1) does not fit int32", fn);
+  EP_REQUIRE_PTR(fn, cnt_e, 4);
+  EP_REQUIRE_PTR(fn, off_pad, 4);
+  EP_REQUIRE_PTR(fn, recv_src_pad, 4);
+  if (T > 0) {
+    EP_REQUIRE_PTR(fn, slot_pos, 4);
+    EP_REQUIRE_PTR(fn, slot_pos_pad, 4);
+  }
+  int n = 0;
+  const cudaError_t e = ep::launch_pad_layout(cnt_e, slot_pos, T, k, E, align, off_pad,
+                                              slot_pos_pad, recv_src_pad,
+                                              static_cast<cudaStream_t>(stream), &n);
   g_launches += n;
   return from_cuda(e, fn);
 }

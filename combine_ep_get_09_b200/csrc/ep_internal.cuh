@@ -85,13 +85,15 @@ struct LayoutArgs {
 size_t layout_workspace_bytes(int T, int k, int E, int R);
 cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s, int *launches);
 
+// n_rows: rows of the receive buffer; slot rows outside [0, n_rows) are
+// skipped.
 cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
-                                 const int32_t *slot_pos, void *recv,
+                                 const int32_t *slot_pos, void *recv, long n_rows,
                                  int num_sms, int32_t *d_err, cudaStream_t s,
                                  int *launches);
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
-                                float *recv_scale, int num_sms, int32_t *d_err,
+                                float *recv_scale, long n_rows, int num_sms, int32_t *d_err,
                                 cudaStream_t s, int *launches);
 // Layout and dispatch in one launch (small batches; see layout_dispatch.cu).
 // layout_dispatch_fusable says whether the sizes (and, for FP8, the scale
@@ -101,10 +103,20 @@ bool layout_dispatch_fusable(int T, int k, int E, int R, int H, bool fp8,
 cudaError_t launch_layout_dispatch(const LayoutArgs &la, const void *x, int H, bool fp8,
                                    void *recv, float *recv_scale, int num_sms, cudaStream_t s,
                                    int *launches);
-cudaError_t launch_combine(const void *y, int T, int H, int k,
+cudaError_t launch_combine(const void *y, long n_rows, int T, int H, int k,
                            const int32_t *slot_pos, const float *w, void *out,
                            int num_sms, int32_t *d_err, cudaStream_t s,
                            int *launches);
+// FP8 expert outputs: e4m3 codes y_q [n_rows, H] and fp32 scales y_scale
+// [n_rows, H / 128].
+cudaError_t launch_combine_fp8(const void *y_q, const float *y_scale, long n_rows, int T,
+                               int H, int k, const int32_t *slot_pos, const float *w,
+                               void *out, int num_sms, int32_t *d_err, cudaStream_t s,
+                               int *launches);
+// Aligned receive segments from a plain layout (pad_layout.cu).
+cudaError_t launch_pad_layout(const int32_t *cnt_e, const int32_t *slot_pos, int T, int k,
+                              int E, int align, int32_t *off_pad, int32_t *slot_pos_pad,
+                              int32_t *recv_src_pad, cudaStream_t s, int *launches);
 
 // Sets the message ep_last_error_string() returns on this host thread and
 // returns `status` (for entry points defined outside ep_abi.cu).

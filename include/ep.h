@@ -133,9 +133,14 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
  * x           [T,H] bf16.
  * slot_pos    [T,k] int32 from ep_get_layout; values outside [0, T*k) are
  *             skipped.
- * recv        [T*k, H] bf16 (fp8 == 0) or e4m3 bytes (fp8 != 0).  Rows no
- *             slot points at are left untouched.
- * recv_scale  [T*k, H/128] fp32 (fp8 != 0, 4-byte aligned), else ignored.
+ * recv        [recv_rows, H] bf16 (fp8 == 0) or e4m3 bytes (fp8 != 0).  Rows
+ *             no slot points at are left untouched.
+ * recv_scale  [recv_rows, H/128] fp32 (fp8 != 0, 4-byte aligned), else
+ *             ignored.
+ * recv_rows   rows of recv (and recv_scale); slot rows outside
+ *             [0, recv_rows) are skipped.  0 means T*k, the size of the
+ *             packed layout; an aligned layout (ep_pad_layout) needs
+ *             ep_aligned_rows(T, k, E, align).
  * T >= 0, 1 <= k <= EP_MAX_K, H > 0 with H % 8 == 0 (H % 128 == 0 for
  * fp8), T*k < 2^31.
  * num_sms     SMs to spread the work over (0 = all of them).
@@ -143,8 +148,8 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
  */
 ep_status_t ep_dispatch(const void *x, int T, int H, int k,
                         const int32_t *slot_pos, int fp8, void *recv,
-                        float *recv_scale, int num_sms, int32_t *d_err,
-                        void *stream);
+                        float *recv_scale, int recv_rows, int num_sms,
+                        int32_t *d_err, void *stream);
 
 /*
  * ep_layout_dispatch -- ep_get_layout followed by ep_dispatch, with the
@@ -185,8 +190,10 @@ ep_status_t ep_layout_dispatch(const void *idx, int idx_is_int64, int T,
  *   acc = 0.0f;  for j = 0..k-1 with slot_pos[t,j] = p >= 0:
  *       acc = fma(w[t,j], float(y[p, :]), acc)
  *   out[t, :] = bf16 round-to-nearest-even(acc)
- * y          [T*k, H] bf16 expert outputs in receive-row order.
- * slot_pos   [T,k] int32; values outside [0, T*k) are skipped.
+ * y          [y_rows, H] bf16 expert outputs in receive-row order.
+ * y_rows     rows of y (0 means T*k); slot rows outside [0, y_rows) are
+ *            skipped.
+ * slot_pos   [T,k] int32 (packed or aligned layout).
  * w          [T,k] fp32 gate weights (4-byte aligned), or NULL for unit
  *            weights: out[t] is then the plain fp32 sum of the kept slot
  *            rows (how per-rank partial outputs combine, see
@@ -194,9 +201,56 @@ ep_status_t ep_layout_dispatch(const void *idx, int idx_is_int64, int T,
  * out        [T,H] bf16; a token with no kept slot gets +0.
  * Limits as ep_dispatch (H % 8 == 0).  num_sms and d_err as ep_dispatch.
  */
-ep_status_t ep_combine(const void *y, int T, int H, int k,
+ep_status_t ep_combine(const void *y, int y_rows, int T, int H, int k,
                        const int32_t *slot_pos, const float *w, void *out,
                        int num_sms, int32_t *d_err, void *stream);
+
+/*
+ * ep_combine_fp8 -- ep_combine for expert outputs kept in the FP8 form of
+ * the dispatch (e4m3 codes plus one fp32 scale per row and 128-channel
+ * block).
+ *
+ * A combine variant beside DeepEP's FP8 dispatch (chinainews.com item,
+ * feature list; Wallstreetcn review of the release): the pages give no
+ * arithmetic for it.  Reading: each value is decoded exactly and scaled in
+ * fp32, then enters the same chain as ep_combine:
+ *   v = fp32_rn(e4m3(y_q[p, c]) * y_scale[p, c / 128])
+ *   acc = fma(w[t,j], v, acc) in slot order from 0.0f; out = bf16_rne(acc)
+ * y_q       [y_rows, H] e4m3 bytes (16-byte aligned).
+ * y_scale   [y_rows, H/128] fp32 (4-byte aligned; 16-byte aligned rows and
+ *           H % 512 == 0 take the bulk-copy kernel).
+ * y_rows, slot_pos, w, out, num_sms, d_err: as ep_combine.  H % 128 == 0.
+ */
+ep_status_t ep_combine_fp8(const void *y_q, const float *y_scale, int y_rows,
+                           int T, int H, int k, const int32_t *slot_pos,
+                           const float *w, void *out, int num_sms,
+                           int32_t *d_err, void *stream);
+
+/*
+ * ep_pad_layout -- receive segments aligned for a grouped GEMM.
+ *
+ * The dispatch layout packs the experts' rows back to back; a grouped GEMM
+ * over the receive buffer in tiles of `align` rows wants each expert's
+ * segment to start on a tile boundary.  The pages describe the layout only
+ * as DeepEP's dispatch target (chinainews.com item, feature list); the
+ * padded form is this library's.  From a layout of ep_get_layout:
+ *   off_pad[e]        = sum_{e' < e} ceil(cnt_e[e'] / align) * align,
+ *                       off_pad[E] = rows in use with padding
+ *   slot_pos_pad[t,j] = off_pad[e] + (slot_pos[t,j] - off_e[e]), or -1
+ *   recv_src_pad[r]   = token of row r; -1 for padding rows and past
+ *                       off_pad[E]
+ * cnt_e        [E] int32 and slot_pos [T,k] int32 from one ep_get_layout.
+ * off_pad      [E+1] int32.  slot_pos_pad [T,k] int32 (may be slot_pos).
+ * recv_src_pad [ep_aligned_rows(T, k, E, align)] int32.
+ * Dispatch and combine then take slot_pos_pad with recv_rows = y_rows =
+ * ep_aligned_rows(T, k, E, align).  T >= 0, k >= 1, 1 <= E <= EP_MAX_E,
+ * align >= 1, T*k + E*(align-1) < 2^31.
+ */
+size_t ep_aligned_rows(int T, int k, int E, int align);
+ep_status_t ep_pad_layout(const int32_t *cnt_e, const int32_t *slot_pos,
+                          int T, int k, int E, int align, int32_t *off_pad,
+                          int32_t *slot_pos_pad, int32_t *recv_src_pad,
+                          void *stream);
 
 /*
  * ep_get_rank_layout -- rows of the rank-deduplicated dispatch: one receive

@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version():
-    assert ep.lib().ep_abi_version() == 3
+    assert ep.lib().ep_abi_version() == 4
 
 
 def test_workspace_sizes():
@@ -80,17 +80,18 @@ def test_layout_rejects(kw, status):
 
 
 @pytest.mark.parametrize("args,status", [
-    ((16, -1, 64, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),
-    ((16, 4, 0, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),
-    ((16, 4, 12, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_UNSUPPORTED),   # H % 8
-    ((16, 4, 64, 2, 16, 1, 16, 16, 0, None, None), ep.EP_ERR_UNSUPPORTED),     # fp8, H % 128
-    ((16, 4, 64, 33, 16, 0, 16, None, 0, None, None), ep.EP_ERR_UNSUPPORTED),  # k > 32
-    ((16, 4, 64, 2, 16, 0, 16, None, -1, None, None), ep.EP_ERR_INVALID_ARG),  # num_sms
-    ((None, 4, 64, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),
-    ((24, 4, 64, 2, 16, 0, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),   # x misaligned
-    ((16, 4, 128, 2, 16, 1, 16, None, 0, None, None), ep.EP_ERR_INVALID_ARG),  # fp8, no scale
-    ((16, 4, 64, 2, 16, 0, 8, None, 0, None, None), ep.EP_ERR_INVALID_ARG),    # recv misaligned
-    ((16, 4, 64, 2, 16, 0, 16, None, 0, 18, None), ep.EP_ERR_INVALID_ARG),     # d_err misaligned
+    ((16, -1, 64, 2, 16, 0, 16, None, 0, 0, None, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 0, 2, 16, 0, 16, None, 0, 0, None, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 4, 12, 2, 16, 0, 16, None, 0, 0, None, None), ep.EP_ERR_UNSUPPORTED),   # H % 8
+    ((16, 4, 64, 2, 16, 1, 16, 16, 0, 0, None, None), ep.EP_ERR_UNSUPPORTED),     # fp8, H % 128
+    ((16, 4, 64, 33, 16, 0, 16, None, 0, 0, None, None), ep.EP_ERR_UNSUPPORTED),  # k > 32
+    ((16, 4, 64, 2, 16, 0, 16, None, 0, -1, None, None), ep.EP_ERR_INVALID_ARG),  # num_sms
+    ((None, 4, 64, 2, 16, 0, 16, None, 0, 0, None, None), ep.EP_ERR_INVALID_ARG),
+    ((24, 4, 64, 2, 16, 0, 16, None, 0, 0, None, None), ep.EP_ERR_INVALID_ARG),   # x misaligned
+    ((16, 4, 128, 2, 16, 1, 16, None, 0, 0, None, None), ep.EP_ERR_INVALID_ARG),  # fp8, no scale
+    ((16, 4, 64, 2, 16, 0, 8, None, 0, 0, None, None), ep.EP_ERR_INVALID_ARG),    # recv misaligned
+    ((16, 4, 64, 2, 16, 0, 16, None, 0, 0, 18, None), ep.EP_ERR_INVALID_ARG),     # d_err misaligned
+    ((16, 4, 64, 2, 16, 0, 16, None, -1, 0, None, None), ep.EP_ERR_INVALID_ARG),  # recv_rows
 ])
 def test_dispatch_rejects(args, status):
     assert ep.lib().ep_dispatch(*args) == status
@@ -98,16 +99,17 @@ def test_dispatch_rejects(args, status):
 
 def test_dispatch_combine_empty_batch_is_a_no_op():
     # T = 0: valid, nothing to do, nothing touched (no device needed)
-    assert ep.lib().ep_dispatch(None, 0, 64, 2, None, 0, None, None, 0, None, None) == ep.EP_OK
-    assert ep.lib().ep_combine(None, 0, 64, 2, None, None, None, 0, None, None) == ep.EP_OK
+    assert ep.lib().ep_dispatch(None, 0, 64, 2, None, 0, None, None, 0, 0, None, None) == ep.EP_OK
+    assert ep.lib().ep_combine(None, 0, 0, 64, 2, None, None, None, 0, None, None) == ep.EP_OK
 
 
 @pytest.mark.parametrize("args,status", [
-    ((None, 4, 64, 2, 16, None, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),  # no y
-    ((16, 4, 64, 2, 16, 18, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),    # w misaligned
-    ((16, 4, 60, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_UNSUPPORTED),
-    ((16, 4, 64, 2, 16, 16, 40, 0, None, None), ep.EP_ERR_INVALID_ARG),    # out misaligned
-    ((16, 4, 64, 2, 16, 16, 16, 0, 2, None), ep.EP_ERR_INVALID_ARG),       # d_err misaligned
+    ((None, 0, 4, 64, 2, 16, None, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),  # no y
+    ((16, 0, 4, 64, 2, 16, 18, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),    # w misaligned
+    ((16, 0, 4, 60, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_UNSUPPORTED),
+    ((16, 0, 4, 64, 2, 16, 16, 40, 0, None, None), ep.EP_ERR_INVALID_ARG),    # out misaligned
+    ((16, 0, 4, 64, 2, 16, 16, 16, 0, 2, None), ep.EP_ERR_INVALID_ARG),       # d_err misaligned
+    ((16, -1, 4, 64, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),  # y_rows
 ])
 def test_combine_rejects(args, status):
     assert ep.lib().ep_combine(*args) == status
@@ -160,6 +162,51 @@ def _layout_dispatch_call(**kw):
 def test_layout_dispatch_rejects(kw, status):
     assert _layout_dispatch_call(**kw) == status
     assert ep.lib().ep_last_error_string().decode()
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, 16, 0, 4, 128, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),   # no codes
+    ((16, None, 0, 4, 128, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),   # no scales
+    ((16, 16, 0, 4, 64, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_UNSUPPORTED),      # H % 128
+    ((16, 16, -1, 4, 128, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),    # y_rows
+    ((24, 16, 0, 4, 128, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),     # codes align
+    ((16, 18, 0, 4, 128, 2, 16, 16, 16, 0, None, None), ep.EP_ERR_INVALID_ARG),     # scale align
+    ((16, 16, 0, 4, 128, 33, 16, 16, 16, 0, None, None), ep.EP_ERR_UNSUPPORTED),    # k > 32
+    ((16, 16, 0, 4, 128, 2, 16, 16, 40, 0, None, None), ep.EP_ERR_INVALID_ARG),     # out align
+])
+def test_combine_fp8_rejects(args, status):
+    assert ep.lib().ep_combine_fp8(*args) == status
+    assert ep.lib().ep_last_error_string().decode()
+
+
+def test_combine_fp8_empty_batch_is_a_no_op():
+    assert ep.lib().ep_combine_fp8(None, None, 0, 0, 128, 2, None, None, None, 0, None,
+                                   None) == ep.EP_OK
+
+
+def test_aligned_rows():
+    assert ep.ep_aligned_rows(4096, 8, 256, 128) == 4096 * 8 + 256 * 127
+    assert ep.ep_aligned_rows(10, 2, 4, 1) == 20
+    assert ep.ep_aligned_rows(0, 2, 4, 3) == 8
+    assert ep.ep_aligned_rows(10, 2, 4, 0) == 0
+    assert ep.ep_aligned_rows(1 << 30, 4, 4, 2) == 0      # does not fit int32
+
+
+@pytest.mark.parametrize("args,status", [
+    ((16, 16, -1, 2, 4, 2, 16, 16, 16, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 16, 4, 0, 4, 2, 16, 16, 16, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 16, 4, 2, 0, 2, 16, 16, 16, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 16, 4, 2, 4, 0, 16, 16, 16, None), ep.EP_ERR_INVALID_ARG),         # align
+    ((16, 16, 4, 2, 2048, 2, 16, 16, 16, None), ep.EP_ERR_UNSUPPORTED),      # E
+    ((16, 16, 1 << 29, 8, 4, 2, 16, 16, 16, None), ep.EP_ERR_UNSUPPORTED),   # rows overflow
+    ((None, 16, 4, 2, 4, 2, 16, 16, 16, None), ep.EP_ERR_INVALID_ARG),       # cnt_e
+    ((16, None, 4, 2, 4, 2, 16, 16, 16, None), ep.EP_ERR_INVALID_ARG),       # slot_pos
+    ((16, 16, 4, 2, 4, 2, None, 16, 16, None), ep.EP_ERR_INVALID_ARG),       # off_pad
+    ((16, 16, 4, 2, 4, 2, 16, 18, 16, None), ep.EP_ERR_INVALID_ARG),         # slot_pos_pad
+    ((16, 16, 4, 2, 4, 2, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),       # recv_src_pad
+])
+def test_pad_layout_rejects(args, status):
+    assert ep.lib().ep_pad_layout(*args) == status
 
 
 def test_read_error_rejects_null():
