@@ -278,28 +278,44 @@ def bench_ours(args, world, rank, device):
     if ep.ep_read_error(st.d_err, stream) != 0:
         raise RuntimeError("the device reported an error during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # timed region: K steps, each bracketed by its own pair of events and
+    # nothing between its kernels, so consecutive kernels keep their
+    # programmatic-dependent-launch overlap (an event between two kernels
+    # would serialise them)
+    step_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(device)
     launches0 = ep.ep_kernel_launches()
     with ClockSampler(device) as clocks, torch.cuda.stream(stream):
         for i in range(args.steps):
             flush()
-            st.run(stream, evs[i])
+            step_evs[i][0].record(stream)
+            st.run(stream)
+            step_evs[i][1].record(stream)
         stream.synchronize()
     torch.cuda.synchronize(device)
     barrier(world)
     launches = ep.ep_kernel_launches() - launches0
     if ep.ep_read_error(st.d_err, stream) != 0:
         raise RuntimeError("the device reported an error in the timed steps")
+    step_ms = [a.elapsed_time(b) for a, b in step_evs]
+    total_ms = max_over_ranks(sum(step_ms), world, device)
 
+    # per-kernel breakdown: the same steps again, with an event between
+    # every two kernels (not part of `value`)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush()
+            st.run(stream, evs[i])
+        stream.synchronize()
     per_kernel = {n: [] for n in KERNELS}
-    step_ms = []
     for e in evs:
         for j, n in enumerate(KERNELS):
             per_kernel[n].append(e[j].elapsed_time(e[j + 1]))
-        step_ms.append(e[0].elapsed_time(e[4]))
-    total_ms = max_over_ranks(sum(step_ms), world, device)
+    evented_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[4]) for e in evs),
+                                world, device)
     kern_ms = {n: max_over_ranks(statistics.mean(v), world, device) for n, v in per_kernel.items()}
 
     peak, peak_kind = measured_peak()
@@ -339,6 +355,7 @@ def bench_ours(args, world, rank, device):
         },
         "frac_of_8TBs": round(value / world / SPEC_HBM_GBS, 4),
         "kernels": kernels,
+        "ms_per_step_with_kernel_events": round(evented_ms, 4),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(dom_gbs / peak, 4),
@@ -353,6 +370,7 @@ def bench_ours(args, world, rank, device):
         result["rank_dedup"] = bench_rank_dedup(ep, st, cfg, device, world)
     if not args.skip_variants:
         result["combine_variants"] = bench_combine_variants(ep, st, cfg, device, world)
+        result["combine_variants"]["replicas"] = bench_replicas(ep, device, world)
     if not args.skip_overlap:
         result["sm_budget_overlap"] = bench_overlap(ep, st, cfg, device, world)
     if not args.skip_e2e:
@@ -507,8 +525,176 @@ def bench_combine_variants(ep, st, cfg, device, world, iters=20, align=128):
     return res
 
 
+def bench_replicas(ep, device, world, iters=20, hot=16, copies=4):
+    """Redundant copies of the busiest experts on the skewed batch: the
+    `hot` most loaded of 256 experts get `copies` copies each (304 physical
+    experts in 8 ranks).  Times the replica mapping kernel and the layout of
+    the physical ids (each alone, flushed L2) and reports the busiest
+    expert's load before and after."""
+    cfg = workloads.CONFIGS["skewed"]
+    batch = workloads.make_batch(cfg, seed=300, H=8)
+    E, R, T, k = cfg.E, cfg.R, cfg.T, cfg.k
+    idx = batch.idx.to(device)
+    load = np.bincount(batch.idx.numpy().reshape(-1), minlength=E)
+    n_rep = np.ones(E, np.int64)
+    n_rep[np.argsort(-load, kind="stable")[:hot]] = copies
+    rep_off = torch.from_numpy(np.concatenate([[0], np.cumsum(n_rep)]).astype(np.int32)).to(device)
+    E_phys = int(n_rep.sum())
+    rep_ids = torch.arange(E_phys, dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device)
+    flush = L2Flush(device)
+    d_err = torch.zeros(1, dtype=torch.int32, device=device)
+    with torch.cuda.stream(stream):
+        L = ep.ep_get_layout(idx, E, R, d_err=d_err, stream=stream)
+        phys = ep.ep_map_replicas(idx, L, rep_off, rep_ids, d_err=d_err, stream=stream)
+        P = ep.ep_get_layout(phys, E_phys, R, d_err=d_err, stream=stream)
+    stream.synchronize()
+    N = T * k
+    calls = {"map_replicas": (lambda: ep.ep_map_replicas(idx, L, rep_off, rep_ids, out=phys,
+                                                         d_err=d_err, stream=stream),
+                              N * (8 + 4 + 4)),
+             "physical_layout": (lambda: ep.ep_get_layout(phys, E_phys, R, out=P, d_err=d_err,
+                                                          stream=stream),
+                                 N * 4 + N * 8 + T * R)}
+    res = {"workload": f"skewed: T={T}, E={E} in R={R}, top-{k}; the {hot} busiest experts "
+                       f"get {copies} copies ({E_phys} physical experts)",
+           "max_load_logical": int(load.max()), "mean_load": round(float(load.mean()), 1),
+           "max_load_physical": int(P.cnt_e.max().item())}
+    for name, (fn, nbytes) in calls.items():
+        evs = []
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                flush()
+                fn()
+            for _ in range(iters):
+                flush()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                evs.append((a, b))
+        stream.synchronize()
+        us = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e3,
+                            world, device)
+        res[name] = {"us": round(us, 2), "bytes": nbytes}
+    if ep.ep_read_error(d_err, stream) != 0:
+        raise RuntimeError("the device reported an error in the replica runs")
+    return res
+
+
 OVERLAP_GEMM = (4096, 7168, 2048)   # M, K, N of the stand-in expert GEMM
 OVERLAP_SMS = (16, 32, 64, 148)
+GREEN_SMS = (16, 32, 48)
+
+
+class GreenPartition:
+    """Two disjoint SM partitions of the device through CUDA green contexts:
+    about `n_comm` SMs for the copy kernels, the rest for the GEMM, each
+    with its own stream.  Work launched into a partition's stream runs on
+    that partition's SMs only.  Read-only towards the device's settings:
+    nothing outlives the process (close() releases everything)."""
+
+    def __init__(self, device, n_comm):
+        from cuda.bindings import driver as drv
+        self.drv = drv
+        self.ok(drv.cuInit(0))
+        dev, = self.ok(drv.cuDeviceGet(torch.device(device).index or 0))
+        res, = self.ok(drv.cuDeviceGetDevResource(
+            dev, drv.CUdevResourceType.CU_DEV_RESOURCE_TYPE_SM))
+        groups, _, rest = self.ok(drv.cuDevSmResourceSplitByCount(1, res, 0, n_comm))
+        self.n_comm = int(groups[0].sm.smCount)
+        self.n_rest = int(rest.sm.smCount)
+        flag = drv.CUgreenCtxCreate_flags.CU_GREEN_CTX_DEFAULT_STREAM
+        nb = drv.CUstream_flags.CU_STREAM_NON_BLOCKING
+        self.ctxs, self.streams, self.events = [], [], []
+        for r in (groups[0], rest):
+            desc, = self.ok(drv.cuDevResourceGenerateDesc([r], 1))
+            g, = self.ok(drv.cuGreenCtxCreate(desc, dev, flag))
+            self.ctxs.append(g)
+            st, = self.ok(drv.cuGreenCtxStreamCreate(g, nb, 0))
+            self.streams.append(st)
+            # an event of the partition's own context marks the end of its work
+            ctx, = self.ok(drv.cuCtxFromGreenCtx(g))
+            self.ok(drv.cuCtxPushCurrent(ctx))
+            ev, = self.ok(drv.cuEventCreate(drv.CUevent_flags.CU_EVENT_DISABLE_TIMING))
+            self.ok(drv.cuCtxPopCurrent())
+            self.events.append(ev)
+        self.comm = torch.cuda.ExternalStream(int(self.streams[0]), device=device)
+        self.comp = torch.cuda.ExternalStream(int(self.streams[1]), device=device)
+
+    def ok(self, r):
+        err = r[0] if isinstance(r, tuple) else r
+        if err != self.drv.CUresult.CUDA_SUCCESS:
+            raise RuntimeError(f"green context: {err}")
+        return r[1:] if isinstance(r, tuple) else ()
+
+    def timed(self, device, comm, comp):
+        """Device microseconds from a start event on a plain stream, which
+        both partitions wait on, until both partitions' work is done."""
+        drv = self.drv
+        s0 = torch.cuda.current_stream(device)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(s0)
+        for st in self.streams:
+            self.ok(drv.cuStreamWaitEvent(st, drv.CUevent(a.cuda_event), 0))
+        if comm is not None:
+            with torch.cuda.stream(self.comm):
+                comm()
+        if comp is not None:
+            with torch.cuda.stream(self.comp):
+                comp()
+        for st, ev in zip(self.streams, self.events):
+            self.ok(drv.cuEventRecord(ev, st))
+            self.ok(drv.cuStreamWaitEvent(drv.CUstream(s0.cuda_stream), ev, 0))
+        b.record(s0)
+        torch.cuda.synchronize(device)
+        return a.elapsed_time(b) * 1e3
+
+    def close(self):
+        drv = self.drv
+        torch.cuda.synchronize()
+        for st in self.streams:
+            drv.cuStreamDestroy(st)
+        for ev in self.events:
+            drv.cuEventDestroy(ev)
+        for g in self.ctxs:
+            drv.cuGreenCtxDestroy(g)
+
+
+def bench_green_overlap(ep, st, device, world, ops, gemm, flush, gemm_full_us, reps=10):
+    """The copy kernels confined to an SM partition beside the GEMM on the
+    other partition (green contexts), against both on all SMs one after the
+    other."""
+    res = {"baseline": "both on all 148 SMs, one after the other", "rows": []}
+    for S in GREEN_SMS:
+        part = GreenPartition(device, S)
+        try:
+            def med(fn):
+                fn()
+                vals = []
+                for _ in range(reps):
+                    torch.cuda.synchronize(device)
+                    flush()
+                    torch.cuda.synchronize(device)
+                    vals.append(fn())
+                return statistics.median(vals)
+            gemm_rest = med(lambda: part.timed(device, None, gemm))
+            row = {"comm_sms": part.n_comm, "gemm_sms": part.n_rest,
+                   "gemm_alone_us": round(max_over_ranks(gemm_rest, world, device), 2)}
+            for name, (op, full_us) in ops.items():
+                alone = med(lambda: part.timed(device, lambda: op(part.n_comm), None))
+                both = med(lambda: part.timed(device, lambda: op(part.n_comm), gemm))
+                alone = max_over_ranks(alone, world, device)
+                both = max_over_ranks(both, world, device)
+                row[name] = {"alone_us": round(alone, 2), "both_us": round(both, 2),
+                             "serial_all_sms_us": round(full_us + gemm_full_us, 2),
+                             "speedup": round((full_us + gemm_full_us) / both, 3)}
+            res["rows"].append(row)
+        finally:
+            part.close()
+    return res
 
 
 def bench_overlap(ep, st, cfg, device, world, reps=10):
@@ -539,11 +725,17 @@ def bench_overlap(ep, st, cfg, device, world, reps=10):
         torch.matmul(A, B, out=Cm)
 
     ops = {
-        "dispatch_bf16": lambda S: ep.ep_dispatch(st.x, st.layout.slot_pos, recv=st.recv,
-                                                  num_sms=S, d_err=st.d_err, stream=s_comm),
-        "combine": lambda S: ep.ep_combine(st.recv, st.layout.slot_pos, st.w, out=st.out,
-                                           num_sms=S, d_err=st.d_err, stream=s_comm),
+        "dispatch_bf16": lambda S, s=None: ep.ep_dispatch(
+            st.x, st.layout.slot_pos, recv=st.recv, num_sms=S, d_err=st.d_err,
+            stream=s_comm if s is None else s),
+        "combine": lambda S, s=None: ep.ep_combine(
+            st.recv, st.layout.slot_pos, st.w, out=st.out, num_sms=S, d_err=st.d_err,
+            stream=s_comm if s is None else s),
     }
+
+    def op_on(op, S):
+        # the current stream (the partition's, inside GreenPartition.timed)
+        op(S, torch.cuda.current_stream(device))
 
     def trial(comm, comp):
         """Device microseconds from a common start until both streams end."""
@@ -572,6 +764,7 @@ def bench_overlap(ep, st, cfg, device, world, reps=10):
     res = {"gemm": {"mkn": [M, K, N], "us": round(max_over_ranks(gemm_us, world, device), 2),
                     "TFLOP/s": round(2 * M * K * N / (gemm_us * 1e-6) / 1e12, 1)},
            "note": "both_us = dispatch or combine and the GEMM on two streams at once"}
+    full = {}
     for name, op in ops.items():
         rows = []
         for S in OVERLAP_SMS:
@@ -582,7 +775,21 @@ def bench_overlap(ep, st, cfg, device, world, reps=10):
             rows.append({"num_sms": S, "alone_us": round(alone, 2), "both_us": round(both, 2),
                          "serial_us": round(alone + gemm_us, 2),
                          "overlap": round((alone + gemm_us) / both, 3)})
+            if S == OVERLAP_SMS[-1]:
+                full[name] = alone
         res[name] = rows
+    # the same with the copy kernels confined to an SM partition (one GPU
+    # only: a failure on one rank must not leave the others in a collective)
+    if world == 1:
+        try:
+            comm_ops = {name: (lambda S, op=op: op_on(op, S), full[name])
+                        for name, op in ops.items()}
+            res["green_contexts"] = bench_green_overlap(ep, st, device, world, comm_ops, gemm,
+                                                        flush, gemm_us)
+        except Exception as e:  # noqa: BLE001 - reported, not fatal
+            res["green_contexts"] = {"error": repr(e)[:300]}
+    else:
+        res["green_contexts"] = {"skipped": "measured with one GPU only"}
     if ep.ep_read_error(st.d_err, s_comm) != 0:
         raise RuntimeError("the device reported an error in the overlap runs")
     return res

@@ -25,6 +25,7 @@ __all__ = ["EPError", "EPLibraryError", "Layout", "RankLayout", "ep_get_layout",
            "ep_get_layout_noalloc", "EP_NOALLOC_SCRATCH_BYTES",
            "ep_dispatch", "ep_combine", "ep_read_error", "ep_layout_dispatch",
            "ep_combine_fp8", "ep_aligned_rows", "ep_pad_layout", "PaddedLayout",
+           "ep_map_replicas",
            "ep_layout_workspace_bytes", "ep_kernel_launches", "lib",
            "EP_OK", "EP_ERR_INVALID_ARG", "EP_ERR_UNSUPPORTED", "EP_ERR_CUDA",
            "EP_ERR_INDEX", "EP_ERR_TIMEOUT", "LIB_PATH"]
@@ -67,6 +68,7 @@ _SIGNATURES = {
     "ep_combine": ([_vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp], _i),
     "ep_combine_fp8": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp], _i),
     "ep_aligned_rows": ([_i, _i, _i, _i], _sz),
+    "ep_map_replicas": ([_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "ep_pad_layout": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
     "ep_read_error": ([_vp, _vp], _i),
     "ep_get_layout_noalloc": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
@@ -383,3 +385,25 @@ def ep_read_error(d_err: torch.Tensor, stream=None) -> int:
     if st == EP_ERR_CUDA:
         _check(st)
     return int(st)
+
+
+def ep_map_replicas(idx: torch.Tensor, layout: Layout, rep_off: torch.Tensor,
+                    rep_ids: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                    d_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Physical expert ids [T, k] (int32) for logical ids ``idx`` with
+    ``layout`` = ep_get_layout(idx, E, R): expert e's slots, in the layout's
+    order, dealt round-robin over its copies ``rep_ids[rep_off[e]:rep_off[e+1]]``."""
+    for name, t in (("idx", idx), ("rep_off", rep_off), ("rep_ids", rep_ids)):
+        _need_cuda(name, t)
+    if rep_off.dtype != torch.int32 or rep_ids.dtype != torch.int32:
+        raise ValueError("rep_off and rep_ids must be int32")
+    T, k = idx.shape
+    E = rep_off.shape[0] - 1
+    if layout.cnt_e.shape[0] != E:
+        raise ValueError("rep_off needs E + 1 entries for the layout's E experts")
+    if out is None:
+        out = torch.empty((T, k), dtype=torch.int32, device=idx.device)
+    _check(lib().ep_map_replicas(_ptr(idx), int(idx.dtype == torch.int64), T, k, E,
+                                 _ptr(layout.slot_pos), _ptr(layout.off_e), _ptr(rep_off),
+                                 _ptr(rep_ids), _ptr(out), _ptr(d_err), _stream(stream)))
+    return out

@@ -401,6 +401,35 @@ ep_status_t ep_combine_fp8(const void *y_q, const float *y_scale, int y_rows, in
   return from_cuda(e, fn);
 }
 
+ep_status_t ep_map_replicas(const void *idx, int idx_is_int64, int T, int k, int E,
+                            const int32_t *slot_pos, const int32_t *off_e,
+                            const int32_t *rep_off, const int32_t *rep_ids, int32_t *phys_idx,
+                            int32_t *d_err, void *stream) {
+  static const char fn[] = "ep_map_replicas";
+  g_err[0] = '\0';
+  if (T < 0) return fail(EP_ERR_INVALID_ARG, "%s: T=%d < 0", fn, T);
+  if (k < 1) return fail(EP_ERR_INVALID_ARG, "%s: k=%d < 1", fn, k);
+  if (E < 1) return fail(EP_ERR_INVALID_ARG, "%s: E=%d < 1", fn, E);
+  if (static_cast<long long>(T) * k > 0x7fffffffLL)
+    return fail(EP_ERR_UNSUPPORTED, "%s: T*k does not fit int32", fn);
+  EP_REQUIRE_PTR(fn, off_e, 4);
+  EP_REQUIRE_PTR(fn, rep_off, 4);
+  EP_REQUIRE_PTR(fn, rep_ids, 4);
+  if (T > 0) {
+    EP_REQUIRE_PTR(fn, idx, idx_is_int64 ? 8 : 4);
+    EP_REQUIRE_PTR(fn, slot_pos, 4);
+    EP_REQUIRE_PTR(fn, phys_idx, 4);
+  }
+  if (d_err != nullptr && !aligned(d_err, 4))
+    return fail(EP_ERR_INVALID_ARG, "%s: d_err is not 4-byte aligned", fn);
+  int n = 0;
+  const cudaError_t e =
+      ep::launch_map_replicas(idx, idx_is_int64 != 0, T, k, E, slot_pos, off_e, rep_off,
+                              rep_ids, phys_idx, d_err, static_cast<cudaStream_t>(stream), &n);
+  g_launches += n;
+  return from_cuda(e, fn);
+}
+
 size_t ep_aligned_rows(int T, int k, int E, int align) {
   if (T < 0 || k < 1 || E < 1 || align < 1) return 0;
   const long long rows = static_cast<long long>(T) * k + static_cast<long long>(E) * (align - 1);

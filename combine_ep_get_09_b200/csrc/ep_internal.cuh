@@ -113,6 +113,11 @@ cudaError_t launch_combine_fp8(const void *y_q, const float *y_scale, long n_row
                                int H, int k, const int32_t *slot_pos, const float *w,
                                void *out, int num_sms, int32_t *d_err, cudaStream_t s,
                                int *launches);
+// Physical expert of every slot from the logical layout (replicas.cu).
+cudaError_t launch_map_replicas(const void *idx, bool int64_ids, int T, int k, int E,
+                                const int32_t *slot_pos, const int32_t *off_e,
+                                const int32_t *rep_off, const int32_t *rep_ids, int32_t *phys,
+                                int32_t *d_err, cudaStream_t s, int *launches);
 // Aligned receive segments from a plain layout (pad_layout.cu).
 cudaError_t launch_pad_layout(const int32_t *cnt_e, const int32_t *slot_pos, int T, int k,
                               int E, int align, int32_t *off_pad, int32_t *slot_pos_pad,

@@ -285,6 +285,33 @@ ep_status_t ep_get_rank_layout(const uint8_t *in_rank, int T, int R,
                                int32_t *rank_row, int32_t *rank_src, void *ws,
                                size_t ws_bytes, void *stream);
 
+/*
+ * ep_map_replicas -- route the slots of busy experts to redundant copies.
+ *
+ * DeepSeek's expert load balancer places extra copies of the experts in
+ * high demand (deepseekaiinsights, Open Source Week overview, "EPLB and
+ * DualPipe"); the page names no rule for which copy serves a token.
+ * Reading: the i-th slot of logical expert e in the dispatch layout's
+ * stable token-major order (i = slot_pos[t,j] - off_e[e]) goes to copy
+ * i mod n_e, so one expert's copies get equal shares to within one slot:
+ *   phys_idx[t,j] = rep_ids[rep_off[e] + i mod (rep_off[e+1] - rep_off[e])]
+ * A dropped slot stays -1; a bad id or an expert without copies is
+ * recorded in d_err (EP_ERR_INDEX) and its slot dropped.  Lay out and
+ * dispatch the physical ids with ep_get_layout(phys_idx, 0, T, k, E_phys,
+ * R_phys, ...) and the rest of the path as usual.
+ *
+ * idx        [T,k] logical ids (int64 or int32, as ep_get_layout).
+ * slot_pos   [T,k] and off_e [E+1] int32 from ep_get_layout of idx.
+ * rep_off    [E+1] int32, nondecreasing; rep_ids [rep_off[E]] int32.
+ * phys_idx   [T,k] int32 physical ids.
+ * T >= 0, k >= 1, E >= 1, T*k < 2^31.
+ */
+ep_status_t ep_map_replicas(const void *idx, int idx_is_int64, int T, int k,
+                            int E, const int32_t *slot_pos,
+                            const int32_t *off_e, const int32_t *rep_off,
+                            const int32_t *rep_ids, int32_t *phys_idx,
+                            int32_t *d_err, void *stream);
+
 /* Size of the scratch array behind ep_get_layout_noalloc (256 KiB). */
 #define EP_NOALLOC_SCRATCH_BYTES (256u * 1024u)
 

@@ -72,6 +72,9 @@ def lib():
             _u8p, _f32p, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             _i32p, _f32p, _u16p]
         L.ep_oracle_combine_fp8.restype = ctypes.c_int
+        L.ep_oracle_map_replicas.argtypes = [
+            _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _i32p, _i32p, _i32p]
+        L.ep_oracle_map_replicas.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -284,3 +287,22 @@ def combine_fp8(yq, ys, slot_pos, w) -> np.ndarray:
     if st:
         raise ValueError("oracle combine_fp8: invalid arguments")
     return out
+
+
+# ------------------------------------------------------------- replicas
+
+def map_replicas(idx, rep_off, rep_ids):
+    """Physical expert of every slot [T, k] (int32, -1 dropped) and the
+    status: logical expert e's slots, in token-major order, dealt
+    round-robin over its copies rep_ids[rep_off[e]:rep_off[e+1]]."""
+    ix = _np(idx, np.int64)
+    off = _np(rep_off, np.int32)
+    ids = _np(rep_ids, np.int32)
+    T, k = ix.shape
+    E = off.shape[0] - 1
+    phys = np.zeros((T, k), np.int32)
+    st = lib().ep_oracle_map_replicas(_ptr(ix, _i64p), T, k, E, _ptr(off, _i32p),
+                                      _ptr(ids, _i32p), _ptr(phys, _i32p))
+    if st == ORACLE_ERR_INVALID_ARG:
+        raise ValueError("oracle map_replicas: invalid arguments")
+    return phys, st

@@ -46,6 +46,12 @@
  *            v = fp32(e4m3 value * scale), rounded to nearest
  *            out[t,:] = bf16_rne( fma chain over j of w[t,j] * v )
  *
+ *   replicas (redundant copies of busy experts, EPLB): logical expert e
+ *            has n_e = rep_off[e+1] - rep_off[e] physical copies
+ *            rep_ids[rep_off[e] .. rep_off[e+1]); the i-th slot choosing e,
+ *            counted in token-major order from 0, goes to copy i mod n_e
+ *            phys[t,j] = rep_ids[rep_off[e] + (i mod n_e)]
+ *
  *   rank layout (the rank-deduplicated form of dispatch: one row per
  *            (token, rank) pair, DeepEP's per-peer sends)
  *            rank_row[t,r] = off_r[r] + #{t' < t : in_rank[t',r]} if
@@ -444,4 +450,39 @@ int ep_oracle_combine_fp8(const uint8_t *yq, const float *ys, long n_rows, int T
     }
     free(acc);
     return EP_ORACLE_OK;
+}
+
+/* ------------------------------------------------------------- replicas */
+
+/* Physical expert of every slot: walk the slots in token-major order and
+ * deal each logical expert's slots round-robin over its copies.  A dropped
+ * slot stays -1; an id outside [-1, E) or an expert without copies is
+ * reported and its slot dropped. */
+int ep_oracle_map_replicas(const int64_t *idx, int T, int k, int E,
+                           const int32_t *rep_off, const int32_t *rep_ids,
+                           int32_t *phys) {
+    if (T < 0 || k <= 0 || E <= 0)
+        return EP_ORACLE_ERR_INVALID_ARG;
+    long *seen = (long *)calloc((size_t)E, sizeof(long));
+    if (!seen)
+        return EP_ORACLE_ERR_INVALID_ARG;
+    int status = EP_ORACLE_OK;
+    for (int t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            const long i = (long)t * k + j;
+            const int64_t e = idx[i];
+            phys[i] = -1;
+            if (e == -1)
+                continue;
+            if (e < -1 || e >= E || rep_off[e + 1] <= rep_off[e]) {
+                status = EP_ORACLE_ERR_INDEX;
+                continue;
+            }
+            const long n = rep_off[e + 1] - rep_off[e];
+            phys[i] = rep_ids[rep_off[e] + seen[e] % n];
+            seen[e] += 1;
+        }
+    }
+    free(seen);
+    return status;
 }

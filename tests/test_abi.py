@@ -209,6 +209,23 @@ def test_pad_layout_rejects(args, status):
     assert ep.lib().ep_pad_layout(*args) == status
 
 
+@pytest.mark.parametrize("args,status", [
+    ((16, 1, -1, 2, 4, 16, 16, 16, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 1, 4, 0, 4, 16, 16, 16, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),
+    ((16, 1, 4, 2, 0, 16, 16, 16, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),
+    ((None, 1, 4, 2, 4, 16, 16, 16, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),  # idx
+    ((20, 1, 4, 2, 4, 16, 16, 16, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),    # int64 align
+    ((16, 1, 4, 2, 4, None, 16, 16, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),  # slot_pos
+    ((16, 1, 4, 2, 4, 16, None, 16, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),  # off_e
+    ((16, 1, 4, 2, 4, 16, 16, None, 16, 16, None, None), ep.EP_ERR_INVALID_ARG),  # rep_off
+    ((16, 1, 4, 2, 4, 16, 16, 16, None, 16, None, None), ep.EP_ERR_INVALID_ARG),  # rep_ids
+    ((16, 1, 4, 2, 4, 16, 16, 16, 16, None, None, None), ep.EP_ERR_INVALID_ARG),  # phys_idx
+    ((16, 1, 4, 2, 4, 16, 16, 16, 16, 16, 2, None), ep.EP_ERR_INVALID_ARG),       # d_err
+])
+def test_map_replicas_rejects(args, status):
+    assert ep.lib().ep_map_replicas(*args) == status
+
+
 def test_read_error_rejects_null():
     assert ep.lib().ep_read_error(None, None) == ep.EP_ERR_INVALID_ARG
 

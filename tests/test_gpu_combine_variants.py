@@ -188,3 +188,65 @@ def test_combine_fp8_special_codes():
                             torch.from_numpy(s).cuda(), torch.from_numpy(slot).cuda(),
                             torch.from_numpy(w).cuda())
     np.testing.assert_array_equal(tensor_bits16(out), oracle.combine_fp8(q, s, slot, w))
+
+
+# -------------------------------------------------------------- replicas
+
+def _replica_table(rng, E, hot, copies):
+    """Logical experts `hot` get `copies` copies each, the rest one; the
+    physical ids are a seeded permutation."""
+    n_rep = np.ones(E, np.int64)
+    n_rep[hot] = copies
+    rep_off = np.concatenate([[0], np.cumsum(n_rep)]).astype(np.int32)
+    rep_ids = rng.permutation(int(rep_off[-1])).astype(np.int32)
+    return rep_off, rep_ids
+
+
+@pytest.mark.parametrize("int32_ids", [False, True])
+def test_replicas_on_the_skewed_workload(int32_ids):
+    # the 16 hottest experts of the Zipf routing get 4 copies: 304 physical
+    # experts in 8 ranks of 38; logical and physical layouts both bit-exact
+    cfg, b = _batch("skewed", 0, H=8)
+    E, R = cfg.E, cfg.R
+    load = np.bincount(b.idx.numpy().reshape(-1), minlength=E)
+    hot = np.argsort(-load, kind="stable")[:16]
+    rng = np.random.default_rng(8)
+    rep_off, rep_ids = _replica_table(rng, E, hot, 4)
+    E_phys = int(rep_off[-1])
+    idx = b.idx.to(torch.int32 if int32_ids else torch.int64).cuda()
+    L = ep.ep_get_layout(idx, E, R)
+    d_err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    phys = ep.ep_map_replicas(idx, L, torch.from_numpy(rep_off).cuda(),
+                              torch.from_numpy(rep_ids).cuda(), d_err=d_err)
+    want, st = oracle.map_replicas(b.idx, rep_off, rep_ids)
+    np.testing.assert_array_equal(phys.cpu().numpy(), want)
+    assert ep.ep_read_error(d_err) == st == ep.EP_OK
+    P = ep.ep_get_layout(phys, E_phys, 8)
+    ref = oracle.layout(torch.from_numpy(want.astype(np.int64)), E_phys, 8)
+    for key in ("cnt_e", "off_e", "slot_pos", "recv_src", "in_rank", "cnt_r"):
+        np.testing.assert_array_equal(getattr(P, key).cpu().numpy().reshape(-1),
+                                      ref[key].reshape(-1), err_msg=key)
+    assert ref["cnt_e"].max() < load.max()        # the hottest load went down
+
+
+def test_replicas_drops_duplicates_bad_ids_and_missing_copies():
+    cfg, b = _batch("decode", 9, T=500, H=8, drop_frac=0.1, dup_frac=0.2)
+    E = cfg.E
+    rng = np.random.default_rng(9)
+    rep_off, rep_ids = _replica_table(rng, E, np.arange(0, E, 5), 3)
+    rep_off = rep_off.copy()
+    # expert 3 has no copy: its slots are reported and dropped
+    n_rep = np.diff(rep_off)
+    n_rep[3] = 0
+    rep_off = np.concatenate([[0], np.cumsum(n_rep)]).astype(np.int32)
+    rep_ids = rep_ids[:int(rep_off[-1])]
+    idx = b.idx.clone()
+    idx[7, 2] = 3
+    idx[9, 0] = 4096                              # bad id
+    L = ep.ep_get_layout(idx.cuda(), E, cfg.R)
+    d_err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    phys = ep.ep_map_replicas(idx.cuda(), L, torch.from_numpy(rep_off).cuda(),
+                              torch.from_numpy(rep_ids).cuda(), d_err=d_err)
+    want, st = oracle.map_replicas(idx, rep_off, rep_ids)
+    np.testing.assert_array_equal(phys.cpu().numpy(), want)
+    assert st == ep.EP_ERR_INDEX and ep.ep_read_error(d_err) == ep.EP_ERR_INDEX

@@ -156,3 +156,56 @@ def test_fp8_dispatch_then_combine_round_trip():
     srow = torch.from_numpy(s[::k].copy()).repeat_interleave(128, dim=1)
     bound = xf.abs() * (2.0 ** -4) * 1.01 + srow * 2.0 ** -9 + got.abs() * 2.0 ** -8
     assert ((got - xf).abs() <= bound).all()
+
+
+# -------------------------------------------------------------- replicas
+
+def test_replicas_one_copy_each_is_a_relabelling():
+    rng = np.random.default_rng(4)
+    T, k, E = 60, 4, 12
+    idx = torch.from_numpy(rng.integers(-1, E, (T, k)).astype(np.int64))
+    perm = rng.permutation(E).astype(np.int32)
+    phys, st = oracle.map_replicas(idx, np.arange(E + 1, dtype=np.int32), perm)
+    want = np.where(idx.numpy() >= 0, perm[np.clip(idx.numpy(), 0, None)], -1)
+    np.testing.assert_array_equal(phys, want)
+    assert st == oracle.ORACLE_OK
+
+
+def test_replicas_hand_case():
+    # expert 0 has copies {5, 3}, expert 1 the single copy {4}; slots of
+    # expert 0 in token-major order: (0,0) (1,1) (2,0) (3,1) -> 5 3 5 3
+    idx = torch.tensor([[0, 1], [1, 0], [0, -1], [1, 0]], dtype=torch.int64)
+    phys, st = oracle.map_replicas(idx, np.array([0, 2, 3], np.int32),
+                                   np.array([5, 3, 4], np.int32))
+    assert phys.tolist() == [[5, 4], [4, 3], [5, -1], [4, 3]]
+    assert st == oracle.ORACLE_OK
+
+
+def test_replicas_balance_and_order_brute_force():
+    # every copy of a logical expert gets floor or ceil of its share, and the
+    # copies are dealt in the order the slots come (checked by enumeration)
+    rng = np.random.default_rng(5)
+    T, k, E = 200, 6, 10
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int64)
+    idx[rng.random(idx.shape) < 0.1] = -1
+    n_rep = rng.integers(1, 5, E)
+    rep_off = np.concatenate([[0], np.cumsum(n_rep)]).astype(np.int32)
+    rep_ids = rng.permutation(int(rep_off[-1])).astype(np.int32)
+    phys, st = oracle.map_replicas(torch.from_numpy(idx), rep_off, rep_ids)
+    assert st == oracle.ORACLE_OK
+    for e in range(E):
+        slots = [(t, j) for t in range(T) for j in range(k) if idx[t, j] == e]
+        copies = rep_ids[rep_off[e]:rep_off[e + 1]]
+        got = [phys[t, j] for t, j in slots]
+        assert got == [copies[i % len(copies)] for i in range(len(slots))]
+        counts = [got.count(c) for c in copies]
+        assert max(counts) - min(counts) <= 1
+    assert ((phys == -1) == (idx == -1)).all()
+
+
+def test_replicas_bad_ids_and_experts_without_copies():
+    idx = torch.tensor([[0, 7], [1, 2]], dtype=torch.int64)
+    phys, st = oracle.map_replicas(idx, np.array([0, 1, 1, 2], np.int32),
+                                   np.array([9, 8], np.int32))
+    assert st == oracle.ORACLE_ERR_INDEX
+    assert phys.tolist() == [[9, -1], [-1, 8]]        # expert 1 has no copy
