@@ -278,44 +278,28 @@ def bench_ours(args, world, rank, device):
     if ep.ep_read_error(st.d_err, stream) != 0:
         raise RuntimeError("the device reported an error during warm-up")
 
-    # timed region: K steps, each bracketed by its own pair of events and
-    # nothing between its kernels, so consecutive kernels keep their
-    # programmatic-dependent-launch overlap (an event between two kernels
-    # would serialise them)
-    step_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
-                for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(device)
     launches0 = ep.ep_kernel_launches()
     with ClockSampler(device) as clocks, torch.cuda.stream(stream):
         for i in range(args.steps):
             flush()
-            step_evs[i][0].record(stream)
-            st.run(stream)
-            step_evs[i][1].record(stream)
+            st.run(stream, evs[i])
         stream.synchronize()
     torch.cuda.synchronize(device)
     barrier(world)
     launches = ep.ep_kernel_launches() - launches0
     if ep.ep_read_error(st.d_err, stream) != 0:
         raise RuntimeError("the device reported an error in the timed steps")
-    step_ms = [a.elapsed_time(b) for a, b in step_evs]
-    total_ms = max_over_ranks(sum(step_ms), world, device)
 
-    # per-kernel breakdown: the same steps again, with an event between
-    # every two kernels (not part of `value`)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            flush()
-            st.run(stream, evs[i])
-        stream.synchronize()
     per_kernel = {n: [] for n in KERNELS}
+    step_ms = []
     for e in evs:
         for j, n in enumerate(KERNELS):
             per_kernel[n].append(e[j].elapsed_time(e[j + 1]))
-    evented_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[4]) for e in evs),
-                                world, device)
+        step_ms.append(e[0].elapsed_time(e[4]))
+    total_ms = max_over_ranks(sum(step_ms), world, device)
     kern_ms = {n: max_over_ranks(statistics.mean(v), world, device) for n, v in per_kernel.items()}
 
     peak, peak_kind = measured_peak()
@@ -355,7 +339,6 @@ def bench_ours(args, world, rank, device):
         },
         "frac_of_8TBs": round(value / world / SPEC_HBM_GBS, 4),
         "kernels": kernels,
-        "ms_per_step_with_kernel_events": round(evented_ms, 4),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(dom_gbs / peak, 4),
@@ -384,8 +367,8 @@ def bench_ours(args, world, rank, device):
 # only reported while these files are byte-for-byte the ones profiled.
 KERNEL_SOURCES = {
     "layout": ("layout.cu", "ep_internal.cuh"),
-    "dispatch_bf16": ("dispatch.cu", "ep_internal.cuh"),
-    "dispatch_fp8": ("dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
+    "dispatch_bf16": ("dispatch_bf16.cu", "ep_internal.cuh"),
+    "dispatch_fp8": ("dispatch_fp8.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
     "combine": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),
     "layout_dispatch_fp8": ("layout_dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
     "combine_fp8": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),

@@ -1,0 +1,69 @@
+// dispatch_bf16.cu -- token rows to expert-contiguous receive rows (bf16).
+//
+// A persistent grid-stride loop over work items (token t, chunk c of its
+// row).  A warp loads the chunk once with 128-bit read-only streaming
+// loads, then writes it to each of the token's k receive rows with
+// coalesced streaming stores, so HBM sees each source byte read once and
+// each destination byte written once.  The slot rows of the token are
+// fetched by lanes 0..k-1 and broadcast with shuffles.
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBf16Vec = 2;  // 16-byte vectors per lane per item
+
+template <int V>
+__global__ void __launch_bounds__(kThreads)
+    dispatch_bf16_kernel(const uint4 *__restrict__ x, int T, int Hv, int k,
+                         const int32_t *__restrict__ slot_pos,
+                         uint4 *__restrict__ recv, long n_rows) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int per_chunk = 32 * V;
+  const int nchunks = (Hv + per_chunk - 1) / per_chunk;
+  const long items = static_cast<long>(T) * nchunks;
+  const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
+  for (long it = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       it < items; it += nwarps) {
+    const int t = static_cast<int>(it / nchunks);
+    const int c = static_cast<int>(it - static_cast<long>(t) * nchunks);
+    const int sp = lane < k ? __ldg(slot_pos + static_cast<long>(t) * k + lane) : -1;
+    const int v0 = c * per_chunk + lane;
+    const uint4 *src = x + static_cast<long>(t) * Hv;
+    uint4 v[V];
+#pragma unroll
+    for (int u = 0; u < V; ++u)
+      v[u] = v0 + 32 * u < Hv ? ld_stream_v4(src + v0 + 32 * u) : make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < k; ++j) {
+      const int row = __shfl_sync(0xffffffffu, sp, j);
+      if (row < 0 || row >= n_rows) continue;  // uniform across the warp
+      uint4 *dst = recv + static_cast<long>(row) * Hv;
+#pragma unroll
+      for (int u = 0; u < V; ++u)
+        if (v0 + 32 * u < Hv) st_stream_v4(dst + v0 + 32 * u, v[u]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
+                                 const int32_t *slot_pos, void *recv, long n_rows,
+                                 int num_sms, int32_t * /*d_err*/, cudaStream_t s,
+                                 int *launches) {
+  const int Hv = H / 8;
+  const long nchunks = (Hv + 32 * kBf16Vec - 1) / (32 * kBf16Vec);
+  const long items = static_cast<long>(T) * nchunks;
+  if (items == 0) return cudaSuccess;
+  auto kern = dispatch_bf16_kernel<kBf16Vec>;
+  const long grid =
+      persistent_grid(reinterpret_cast<const void *>(kern), kThreads, 0, items, num_sms);
+  ++*launches;
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, s, 1, static_cast<const uint4 *>(x), T,
+                    Hv, k, slot_pos, static_cast<uint4 *>(recv), n_rows);
+}
+
+}  // namespace ep

@@ -1,12 +1,8 @@
-// dispatch.cu -- token rows to expert-contiguous receive rows, as bf16 or
-// with the FP8 (e4m3, per-token per-128-channel fp32 scale) cast fused in.
-//
-// Both kernels are persistent grid-stride loops over work items
-// (token t, chunk c of its row).  A warp loads the chunk once with 128-bit
-// read-only streaming loads, then writes it to each of the token's k receive
-// rows with coalesced streaming stores, so HBM sees each source byte read
-// once and each destination byte written once.  The slot rows of the token
-// are fetched by lanes 0..k-1 and broadcast with shuffles.
+// dispatch_fp8.cu -- token rows to expert-contiguous receive rows with the
+// FP8 cast (e4m3 codes, one fp32 scale per token and 128-channel block)
+// fused in: a bulk-copy kernel for hidden sizes that are multiples of 512
+// and a register kernel for the other multiples of 128.  Both read each
+// source byte once and write each destination byte once.
 #include "bulk.cuh"
 #include "ep_internal.cuh"
 #include "fp8.cuh"
@@ -14,45 +10,15 @@
 namespace ep {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kBf16Vec = 2;  // 16-byte vectors per lane per item (bf16 path)
-
-template <int V>
-__global__ void __launch_bounds__(kThreads)
-    dispatch_bf16_kernel(const uint4 *__restrict__ x, int T, int Hv, int k,
-                         const int32_t *__restrict__ slot_pos,
-                         uint4 *__restrict__ recv, long n_rows) {
-  pdl_trigger();
-  pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int per_chunk = 32 * V;
-  const int nchunks = (Hv + per_chunk - 1) / per_chunk;
-  const long items = static_cast<long>(T) * nchunks;
-  const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
-  for (long it = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       it < items; it += nwarps) {
-    const int t = static_cast<int>(it / nchunks);
-    const int c = static_cast<int>(it - static_cast<long>(t) * nchunks);
-    const int sp = lane < k ? __ldg(slot_pos + static_cast<long>(t) * k + lane) : -1;
-    const int v0 = c * per_chunk + lane;
-    const uint4 *src = x + static_cast<long>(t) * Hv;
-    uint4 v[V];
-#pragma unroll
-    for (int u = 0; u < V; ++u)
-      v[u] = v0 + 32 * u < Hv ? ld_stream_v4(src + v0 + 32 * u) : make_uint4(0, 0, 0, 0);
-    for (int j = 0; j < k; ++j) {
-      const int row = __shfl_sync(0xffffffffu, sp, j);
-      if (row < 0 || row >= n_rows) continue;  // uniform across the warp
-      uint4 *dst = recv + static_cast<long>(row) * Hv;
-#pragma unroll
-      for (int u = 0; u < V; ++u)
-        if (v0 + 32 * u < Hv) st_stream_v4(dst + v0 + 32 * u, v[u]);
-    }
-  }
-}
+constexpr int kThreads = 256;  // register kernel
 
 constexpr int kFp8BulkThreads = 256;
 constexpr int kFp8BulkStages = 2;  // input rows in flight per CTA
+// Cast rows whose bulk stores may still be reading them.  Two (the cast of
+// one token overlapping the stores of the previous one) measured slower at
+// the prefill shape (58.5 vs 54 us alone): the extra stage costs a CTA per
+// SM (5 instead of 6), which hurts more than the overlap helps.
+constexpr int kFp8OutStages = 1;
 
 // FP8 dispatch through shared memory, one whole token row per item (H a
 // multiple of 512, so both the e4m3 row and its H/128 scales are whole
@@ -67,9 +33,9 @@ __global__ void __launch_bounds__(kFp8BulkThreads)
                              float *__restrict__ recv_scale, long n_rows, int32_t *d_err) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int in_bytes = 2 * H, q_bytes = H, nb = H >> 7, s_bytes = 4 * nb;
+  const int out_bytes = q_bytes + s_bytes;                           // a multiple of 16
   unsigned char *in_buf = smem_raw;                                  // [stages][2H]
-  unsigned char *out_q = smem_raw + kFp8BulkStages * in_bytes;       // [H]
-  float *out_s = reinterpret_cast<float *>(out_q + q_bytes);         // [H / 128]
+  unsigned char *out_buf = smem_raw + kFp8BulkStages * in_bytes;     // [out stages][H + H/32]
   __shared__ __align__(8) uint64_t full[kFp8BulkStages];
   __shared__ int rows[2][EP_MAX_K];
   __shared__ int timed_out;
@@ -99,9 +65,13 @@ __global__ void __launch_bounds__(kFp8BulkThreads)
   for (; i < n_mine; ++i) {
     const long t = first + i;
     const int s = static_cast<int>(i % kFp8BulkStages);
+    unsigned char *out_q = out_buf + (i % kFp8OutStages) * out_bytes;
+    float *out_s = reinterpret_cast<float *>(out_q + q_bytes);
     if (tid == 0) {
       if (i + kFp8BulkStages - 1 < n_mine) issue(i + kFp8BulkStages - 1);
-      bulk_wait_read<0>();  // the previous token's stores have left the output stage
+      // the stores of the token that last used this output stage have
+      // read it
+      bulk_wait_read<kFp8OutStages - 1>();
     }
     if (tid < k) rows[i & 1][tid] = __ldg(slot_pos + t * k + tid);
     if (!mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kFp8BulkStages) & 1)))
@@ -211,26 +181,10 @@ __global__ void __launch_bounds__(kThreads)
 
 }  // namespace
 
-cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
-                                 const int32_t *slot_pos, void *recv, long n_rows,
-                                 int num_sms, int32_t * /*d_err*/, cudaStream_t s,
-                                 int *launches) {
-  const int Hv = H / 8;
-  const long nchunks = (Hv + 32 * kBf16Vec - 1) / (32 * kBf16Vec);
-  const long items = static_cast<long>(T) * nchunks;
-  if (items == 0) return cudaSuccess;
-  auto kern = dispatch_bf16_kernel<kBf16Vec>;
-  const long grid =
-      persistent_grid(reinterpret_cast<const void *>(kern), kThreads, 0, items, num_sms);
-  ++*launches;
-  return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, s, 1, static_cast<const uint4 *>(x), T,
-                    Hv, k, slot_pos, static_cast<uint4 *>(recv), n_rows);
-}
-
 // Largest hidden size the bulk FP8 kernel stages in shared memory.
 constexpr int kFp8BulkMaxH = 16384;
 
-int fp8_bulk_smem(int H) { return kFp8BulkStages * 2 * H + H + H / 32; }
+int fp8_bulk_smem(int H) { return kFp8BulkStages * 2 * H + kFp8OutStages * (H + H / 32); }
 
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,

@@ -1,7 +1,8 @@
 // ep_abi.cu -- the extern "C" entry points of libep.so: argument checks,
 // launch, error reporting.  Every check happens before anything is
-// enqueued; the kernels themselves live in layout.cu, dispatch.cu and
-// combine.cu.
+// enqueued; the kernels live in layout.cu, layout_dispatch.cu,
+// dispatch_bf16.cu, dispatch_fp8.cu, combine.cu, pad_layout.cu and
+// replicas.cu.
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>

@@ -112,9 +112,9 @@ cudaError_t launch_pad_layout(const int32_t *cnt_e, const int32_t *slot_pos, int
   const long n_cap = static_cast<long>(T) * k + static_cast<long>(E) * (align - 1);
   const int smem = (3 * E + 2) * static_cast<int>(sizeof(int));
   const long work = n_cap > static_cast<long>(T) * k ? n_cap : static_cast<long>(T) * k;
-  // about 4 elements per thread, at most the CTAs that fit at once
+  // about 2 elements per thread, at most the CTAs that fit at once
   const long grid = persistent_grid(reinterpret_cast<const void *>(pad_layout_kernel),
-                                    kPadThreads, smem, (work + 127) / 128, 0);
+                                    kPadThreads, smem, (work + 63) / 64, 0);
   ++*launches;
   return launch_pdl(pad_layout_kernel, dim3(grid > 0 ? grid : 1), dim3(kPadThreads), smem, s, 1,
                     cnt_e, slot_pos, T, k, E, align, off_pad, slot_pos_pad, recv_src_pad, n_cap);

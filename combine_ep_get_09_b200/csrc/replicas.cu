@@ -53,14 +53,14 @@ cudaError_t launch_map_replicas(const void *idx, bool int64_ids, int T, int k, i
   if (int64_ids) {
     auto kern = map_replicas_kernel<long long>;
     const long grid = persistent_grid(reinterpret_cast<const void *>(kern), kRepThreads, 0,
-                                      (n + 127) / 128, 0);
+                                      (n + 31) / 32, 0);
     return launch_pdl(kern, dim3(grid), dim3(kRepThreads), 0, s, 1,
                       static_cast<const long long *>(idx), n, E, slot_pos, off_e, rep_off,
                       rep_ids, phys, d_err);
   }
   auto kern = map_replicas_kernel<int32_t>;
   const long grid = persistent_grid(reinterpret_cast<const void *>(kern), kRepThreads, 0,
-                                    (n + 127) / 128, 0);
+                                    (n + 31) / 32, 0);
   return launch_pdl(kern, dim3(grid), dim3(kRepThreads), 0, s, 1,
                     static_cast<const int32_t *>(idx), n, E, slot_pos, off_e, rep_off, rep_ids,
                     phys, d_err);

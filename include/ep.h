@@ -3,14 +3,15 @@
  * library (libep.so).
  *
  * The operation is DeepEP's: route every token to the experts of its top-k
- * choice and bring the expert outputs back ("all-to-all" dispatch and
- * combine for MoE, with native FP8 dispatch -- chinainews.com, "DeepSeek
- * releases DeepEP", feature list; Wallstreetcn/lbkrs review, feature list;
- * dataforcee.us rewrite, "Technological Views and Benefits": tokens are
- * "shipped and combined" across experts).  Here the expert-parallel ranks
- * are logical partitions of one GPU's memory: rank r owns the G = E / R
- * consecutive experts [r*G, (r+1)*G), and "sending to rank r" means writing
- * into rank r's segment of one expert-contiguous receive buffer.
+ * choice and bring the expert outputs back (all-to-all dispatch and
+ * combine for MoE, with FP8 dispatch -- chinainews.com, "DeepSeek releases
+ * DeepEP", feature list; Wallstreetcn/lbkrs review, feature list;
+ * dataforcee.us rewrite, "Technological Views and Benefits": tokens travel
+ * to their experts and the results are merged back).  Here the
+ * expert-parallel ranks are logical partitions of one GPU's memory: rank r
+ * owns the G = E / R consecutive experts [r*G, (r+1)*G), and "sending to
+ * rank r" means writing into rank r's segment of one expert-contiguous
+ * receive buffer.
  *
  * Notation: T tokens, hidden size H, top-k slots per token, E experts,
  * R ranks.  idx[T,k] expert ids (-1 = dropped slot), w[T,k] fp32 gate
@@ -119,10 +120,9 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
 /*
  * ep_dispatch -- send each token to its experts' receive rows.
  *
- * DeepEP's dispatch (chinainews.com item, feature list: "all-to-all" for
- * MoE, native FP8 support; Wallstreetcn/lbkrs review: "Native FP8 dispatch
- * support"; frogred8 blog, TMA bulk copies and read-only non-coherent
- * loads).  For every slot (t,j) with slot_pos[t,j] = p >= 0:
+ * DeepEP's dispatch (chinainews.com item, feature list: all-to-all for
+ * MoE, FP8 support; Wallstreetcn/lbkrs review, feature list: FP8 dispatch;
+ * frogred8 blog, TMA bulk copies and read-only non-coherent loads).  For every slot (t,j) with slot_pos[t,j] = p >= 0:
  *   fp8 == 0:  recv[p, :] = x[t, :]                    (bf16 rows)
  *   fp8 != 0:  per 128-channel block b of token t,
  *              a = max |x[t, 128b : 128b+128]| (NaN propagates),

@@ -11,8 +11,8 @@
  * What the path computes comes from the DeepEP pages (the chinainews.com
  * item "DeepSeek releases DeepEP", feature list: all-to-all dispatch and
  * combine for MoE, native FP8 dispatch; the dataforcee.us rewrite, section
- * "Technological Views and Benefits": tokens are "shipped and combined"
- * across experts; the frogred8 blog, section "Implementation of SMs
+ * "Technological Views and Benefits": tokens travel to their experts and
+ * the results are merged back; the frogred8 blog, section "Implementation of SMs
  * dedicated to network communication": per-rank senders, up to 8 NVLink
  * peers).  The pages give no formula, so the plain reading used here is:
  *
