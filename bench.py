@@ -366,22 +366,27 @@ def bench_ours(args, world, rank, device):
 # Library sources each kernel is built from: a profile's DRAM traffic is
 # only reported while these files are byte-for-byte the ones profiled.
 KERNEL_SOURCES = {
-    "layout": ("layout.cu", "ep_internal.cuh"),
-    "dispatch_bf16": ("dispatch_bf16.cu", "ep_internal.cuh"),
-    "dispatch_fp8": ("dispatch_fp8.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
-    "combine": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),
-    "layout_dispatch_fp8": ("layout_dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_internal.cuh"),
-    "combine_fp8": ("combine.cu", "bulk.cuh", "ep_internal.cuh"),
+    "layout": ("layout.cu", "ep_device.cuh"),
+    "dispatch_bf16": ("dispatch_bf16.cu", "ep_device.cuh"),
+    "dispatch_fp8": ("dispatch_fp8.cu", "fp8.cuh", "bulk.cuh", "ep_device.cuh"),
+    "combine": ("combine.cu", "bulk.cuh", "ep_device.cuh"),
+    "layout_dispatch_fp8": ("layout_dispatch.cu", "fp8.cuh", "bulk.cuh", "ep_device.cuh"),
+    "combine_fp8": ("combine.cu", "bulk.cuh", "ep_device.cuh"),
 }
 
 
 def kernel_source_digest(kernel: str) -> str:
+    """sha256 over the files a kernel's device code is built from, plus the
+    constants of the public header (its #define lines; its comments do not
+    change a kernel)."""
     import hashlib
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "combine_ep_get_09_b200", "csrc", name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
+    with open(os.path.join(ROOT, "include", "ep.h")) as f:
+        h.update("".join(l for l in f if l.startswith("#define")).encode())
     return h.hexdigest()
 
 
