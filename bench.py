@@ -375,16 +375,24 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments and blank lines (comments do not
+    change a compiled kernel)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
+
+
 def kernel_source_digest(kernel: str) -> str:
-    """sha256 over the files a kernel's device code is built from, plus the
-    constants of the public header (its #define lines; its comments do not
-    change a kernel)."""
+    """sha256 over the code (comments stripped) of the files a kernel's
+    device code is built from, plus the #define constants of the public
+    header."""
     import hashlib
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "combine_ep_get_09_b200", "csrc", name), "rb") as f:
+        with open(os.path.join(ROOT, "combine_ep_get_09_b200", "csrc", name)) as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     with open(os.path.join(ROOT, "include", "ep.h")) as f:
         h.update("".join(l for l in f if l.startswith("#define")).encode())
     return h.hexdigest()

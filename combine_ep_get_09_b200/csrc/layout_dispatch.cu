@@ -5,18 +5,14 @@
 // (dataforcee.us rewrite, "Technological Views and Benefits": 128 tokens,
 // eight experts).  Inside one GPU such a step is bound by launch and
 // dependency latency, not by bytes, so this path drops the layout launch
-// and the wait between it and the dispatch: every CTA computes the whole
-// layout of the batch in its own shared memory from the ids (a few KB,
-// served by L2 after the first CTA reads them), with no CTA ever waiting on
-// another, then dispatches its own contiguous range of tokens and writes
-// the layout entries of those tokens; CTA 0 also writes the counts and
-// offsets.
-//
-// Inside a CTA the work that does not need the layout runs beside it: the
-// token rows are bulk-loaded (cp.async.bulk) as the kernel starts, and
-// while warps 0..7 build the layout the other warps cast the first row to
-// FP8.  Once both are done, the receive rows are known and k threads issue
-// the bulk stores of the row, one receive row each.
+// and the wait between it and the dispatch: every CTA works out the
+// layout entries it needs from the ids themselves (a few KB, served by L2
+// after the first CTA reads them), with no CTA ever waiting on another,
+// then dispatches its own tokens and writes their layout entries.  The
+// token rows are bulk-loaded (cp.async.bulk) as the kernel starts, and the
+// FP8 cast, which does not need the layout, runs while the layout work is
+// in flight.  Results are bit-identical to ep_get_layout followed by
+// ep_dispatch.
 //
 // Two kernels:
 //  * layout_dispatch_token_kernel (T + 1 CTAs fit on the GPU at once, e.g.
@@ -26,19 +22,20 @@
 //    major, token-major inside an expert -- the stable order of the unfused
 //    layout, duplicates included.  The CTA counts those keys over all ids
 //    (each thread a strided share, a warp-wide sum, one shared atomic per
-//    warp and slot), so it needs no table, no scan and no zeroing; CTA T
-//    alone builds the per-expert and per-rank counts and offsets.
+//    warp and slot), so it needs no table, no scan and no zeroing; it casts
+//    its row while the ids are in flight.  CTA T alone builds the
+//    per-expert and per-rank counts and offsets.
 //  * layout_dispatch_kernel (larger batches): CTAs own contiguous token
-//    ranges and each builds the token-set table below.
-//
-// The layout in shared memory is one token bit set per expert: bit t % 32
-// of mask[e][t / 32] is set when token t chose expert e.  The receive row
-// of slot (t, j) with expert e is off_e[e] + (tokens before t that chose e),
-// a popcount of the set below bit t -- the stable token-major order of the
-// unfused layout.  A token naming one expert twice (two slots, as the
-// unfused path accepts) is seen while the sets are built; the ranks are
-// then counted over the flat slot order instead.  Results are bit-identical
-// to ep_get_layout followed by ep_dispatch.
+//    ranges.  Warps 0..7 of every CTA build the whole layout in shared
+//    memory as one token bit set per expert (bit t % 32 of mask[e][t / 32]
+//    set when token t chose expert e), per-expert counts and their scan;
+//    meanwhile warps 8..23 cast the CTA's first row.  The receive row of
+//    slot (t, j) with expert e is off_e[e] + (tokens before t that chose
+//    e), a popcount of the set below bit t.  A token naming one expert
+//    twice (two slots, as the unfused path accepts) is seen while the sets
+//    are built; the ranks are then counted over the flat slot order
+//    instead.  CTA 0 writes the counts and offsets; k threads issue each
+//    token's bulk stores, one receive row each.
 #include <cuda_bf16.h>
 
 #include "bulk.cuh"

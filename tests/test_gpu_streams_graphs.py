@@ -57,6 +57,11 @@ class Path:
             self.idx.copy_(b.idx, non_blocking=True)
             self.x.copy_(b.x, non_blocking=True)
             self.w.copy_(b.w, non_blocking=True)
+            # rows no slot points at are left untouched by dispatch; start
+            # them at zero like the oracle's buffers
+            self.recv.zero_()
+            self.q.view(torch.uint8).zero_()
+            self.s.zero_()
 
     def run(self, stream):
         c = self.cfg
