@@ -21,8 +21,9 @@
 //    (expert, flat slot index) key is smaller than (e, b*k + j): expert-
 //    major, token-major inside an expert -- the stable order of the unfused
 //    layout, duplicates included.  The CTA counts those keys over all ids
-//    (each thread a strided share, a warp-wide sum, one shared atomic per
-//    warp and slot), so it needs no table, no scan and no zeroing; it casts
+//    (each thread a strided share, a warp-wide sum per slot, then the
+//    warps' sums added by one thread per slot), so it needs no table, no
+//    scan and no zeroing; it casts
 //    its row while the ids are in flight.  CTA T alone builds the
 //    per-expert and per-rank counts and offsets.
 //  * layout_dispatch_kernel (larger batches): CTAs own contiguous token
@@ -388,11 +389,11 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(const FusedAr
 
 // ------------------------------------------------ one token per CTA
 
-constexpr int kTokThreads = 512;
+constexpr int kTokThreads = 1024;
 constexpr int kTokWarps = kTokThreads / kWarp;
 constexpr int kTokIdBatch = 4;  // ids per thread loaded before the cast
 
-__host__ __device__ inline SmemMap token_smem_map(int T, int k, int E, int R, int H, bool fp8) {
+__host__ __device__ inline SmemMap token_smem_map(int T, int k, int E, int H, bool fp8) {
   SmemMap m;
   int o = 0;
   m.in = o;     o += 2 * H;
@@ -401,7 +402,7 @@ __host__ __device__ inline SmemMap token_smem_map(int T, int k, int E, int R, in
   m.mask = o;   // unused
   m.cnt = o;    o += align16(static_cast<long>(E) * 4);
   m.off = o;    o += align16(static_cast<long>(E + 1) * 4);
-  m.cnt_r = o;  o += align16(static_cast<long>(R) * 4);
+  m.cnt_r = o;  // unused: per-rank counts come from ballots
   m.ids = o;    o += align16(static_cast<long>(T) * k * 2);
   m.rows = o;
   m.total = o;
@@ -440,16 +441,16 @@ __device__ void token_cta_exclusive_scan(const int *in, int *out, int n, int *wa
 template <typename IdT, bool kFp8>
 __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(const FusedArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const SmemMap sm = token_smem_map(a.T, a.k, a.E, a.R, a.H, kFp8);
+  const SmemMap sm = token_smem_map(a.T, a.k, a.E, a.H, kFp8);
   unsigned char *in_buf = smem + sm.in;
   uint2 *out_q = reinterpret_cast<uint2 *>(smem + sm.out_q);
   float *out_s = reinterpret_cast<float *>(smem + sm.out_s);
   int *cnt = reinterpret_cast<int *>(smem + sm.cnt);
   int *off = reinterpret_cast<int *>(smem + sm.off);
-  int *cnt_r = reinterpret_cast<int *>(smem + sm.cnt_r);
   int16_t *ids = reinterpret_cast<int16_t *>(smem + sm.ids);
   __shared__ __align__(8) uint64_t full;
-  __shared__ int rank_sm[EP_MAX_K];
+  __shared__ int part[kTokWarps][EP_MAX_K];   // per-warp counts of smaller keys
+  __shared__ int rpart[kTokWarps][EP_MAX_R];  // counts CTA: per-warp tokens per rank
   __shared__ int warp_tot[kTokWarps];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -464,12 +465,8 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
     mbar_init(&full, 1);
     mbar_init_fence();
   }
-  if (counts_cta) {
+  if (counts_cta)
     for (int q = tid; q < E; q += kTokThreads) cnt[q] = 0;
-    for (int q = tid; q < R; q += kTokThreads) cnt_r[q] = 0;
-  } else if (tid < EP_MAX_K) {
-    rank_sm[tid] = 0;
-  }
   __syncthreads();  // barrier initialised and counters zeroed before use
   pdl_wait();       // ids and the row come from the previous kernel on the stream
   if (tid == 0 && !counts_cta) {
@@ -519,16 +516,21 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
   }
 
   if (counts_cta) {
-    // 2c. the counts and offsets of the whole batch
-    for (int tt = tid; tt < T; tt += kTokThreads) {
-      unsigned long long rm = 0ull;  // ranks of token tt's kept slots (R <= 64)
-      for (int j = 0; j < k; ++j) {
-        const int e = ids[tt * k + j];
-        if (e >= 0) rm |= 1ull << ((static_cast<unsigned long long>(e) * a.g_magic) >> 32);
-      }
-      while (rm != 0ull) {
-        atomicAdd(&cnt_r[__ffsll(static_cast<long long>(rm)) - 1], 1);
-        rm &= rm - 1ull;
+    // 2c. the counts and offsets of the whole batch; tokens per rank as one
+    //     ballot per rank and warp over the tokens' rank masks (R <= 64)
+    if (lane == 0)
+      for (int r = 0; r < R; ++r) rpart[warp][r] = 0;
+    for (int t0 = 0; t0 < T; t0 += kTokThreads) {  // same trip count in every lane
+      const int tt = t0 + tid;
+      unsigned long long rm = 0ull;
+      if (tt < T)
+        for (int j = 0; j < k; ++j) {
+          const int e = ids[tt * k + j];
+          if (e >= 0) rm |= 1ull << ((static_cast<unsigned long long>(e) * a.g_magic) >> 32);
+        }
+      for (int r = 0; r < R; ++r) {
+        const unsigned bal = __ballot_sync(0xffffffffu, ((rm >> r) & 1ull) != 0ull);
+        if (lane == 0) rpart[warp][r] += __popc(bal);
       }
     }
     token_cta_exclusive_scan(cnt, off, E, warp_tot);
@@ -543,7 +545,9 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
       int carry = 0;
       for (int b = 0; b < R; b += 32) {
         const int r = b + lane;
-        const int c = r < R ? cnt_r[r] : 0;
+        int c = 0;
+        if (r < R)
+          for (int v = 0; v < kTokWarps; ++v) c += rpart[v][r];
         const int incl = warp_incl_scan(c);
         if (r < R) {
           a.cnt_r[r] = c;
@@ -576,7 +580,7 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
       const int sum = __reduce_add_sync(0xffffffffu, c[jj]);
-      if (lane == 0 && sum != 0 && j0 + jj < k) atomicAdd(&rank_sm[j0 + jj], sum);
+      if (lane == 0 && j0 + jj < k) part[warp][j0 + jj] = sum;
     }
   }
   __syncthreads();
@@ -591,7 +595,9 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
     }
   }
   if (warp == 0 && lane < k) {
-    const int row = ids[f0 + lane] >= 0 ? rank_sm[lane] : -1;
+    int before = 0;
+    for (int v = 0; v < kTokWarps; ++v) before += part[v][lane];
+    const int row = ids[f0 + lane] >= 0 ? before : -1;
     a.slot_pos[f0 + lane] = row;
     if (row >= 0) {
       a.recv_src[row] = t;
@@ -611,7 +617,7 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
 template <typename IdT, bool kFp8>
 cudaError_t launch_token_kernel(const FusedArgs &a, cudaStream_t s) {
   auto kern = layout_dispatch_token_kernel<IdT, kFp8>;
-  const int smem = token_smem_map(a.T, a.k, a.E, a.R, a.H, kFp8).total;
+  const int smem = token_smem_map(a.T, a.k, a.E, a.H, kFp8).total;
   const cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
   if (err != cudaSuccess) return err;
   return launch_pdl(kern, dim3(a.T + 1), dim3(kTokThreads), smem, s, 1, a);
@@ -620,7 +626,7 @@ cudaError_t launch_token_kernel(const FusedArgs &a, cudaStream_t s) {
 // CTAs of the token kernel that fit on `num_sms` SMs at once (0 = all).
 template <typename IdT, bool kFp8>
 long token_kernel_capacity(const FusedArgs &a, int num_sms) {
-  const int smem = token_smem_map(a.T, a.k, a.E, a.R, a.H, kFp8).total;
+  const int smem = token_smem_map(a.T, a.k, a.E, a.H, kFp8).total;
   return persistent_grid(reinterpret_cast<const void *>(layout_dispatch_token_kernel<IdT, kFp8>),
                          kTokThreads, smem, 1L << 40, num_sms);
 }

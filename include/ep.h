@@ -59,7 +59,7 @@ typedef int ep_status_t;
 #define EP_MAX_E 1024  /* experts                          */
 #define EP_MAX_R 64    /* logical ranks                    */
 
-/* Version of this ABI (incremented on any signature change): 2. */
+/* Version of this ABI (incremented on any signature change): 4. */
 int ep_abi_version(void);
 
 /* Message of the last error returned on this host thread ("" if none). */
@@ -122,7 +122,8 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
  *
  * DeepEP's dispatch (chinainews.com item, feature list: all-to-all for
  * MoE, FP8 support; Wallstreetcn/lbkrs review, feature list: FP8 dispatch;
- * frogred8 blog, TMA bulk copies and read-only non-coherent loads).  For every slot (t,j) with slot_pos[t,j] = p >= 0:
+ * frogred8 blog, TMA bulk copies and read-only non-coherent loads).  For
+ * every slot (t,j) with slot_pos[t,j] = p >= 0:
  *   fp8 == 0:  recv[p, :] = x[t, :]                    (bf16 rows)
  *   fp8 != 0:  per 128-channel block b of token t,
  *              a = max |x[t, 128b : 128b+128]| (NaN propagates),
@@ -131,8 +132,8 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
  *              nearest; e4m3 round-to-nearest-even, saturating to +-448;
  *              NaN -> 0x7f);  recv_scale[p, b] = s.
  * x           [T,H] bf16.
- * slot_pos    [T,k] int32 from ep_get_layout; values outside [0, T*k) are
- *             skipped.
+ * slot_pos    [T,k] int32 from ep_get_layout (or ep_pad_layout); values
+ *             outside [0, recv_rows) are skipped.
  * recv        [recv_rows, H] bf16 (fp8 == 0) or e4m3 bytes (fp8 != 0).  Rows
  *             no slot points at are left untouched.
  * recv_scale  [recv_rows, H/128] fp32 (fp8 != 0, 4-byte aligned), else
@@ -160,10 +161,12 @@ ep_status_t ep_dispatch(const void *x, int T, int H, int k,
  * (dataforcee.us rewrite, "Technological Views and Benefits": 128 tokens,
  * eight experts); on one GPU their cost is launch and dependency latency.
  * When T*k <= 8192, E * ceil(T/32) * 4 <= 32 KiB and H <= 16384 (for FP8
- * also H % 512 == 0 and a 16-byte aligned recv_scale), one kernel computes
- * the layout redundantly in every CTA's shared memory, writes it, and
- * dispatches; otherwise the call enqueues the two kernels of ep_get_layout
- * and ep_dispatch (ep_kernel_launches tells which ran).
+ * also H % 512 == 0 and a 16-byte aligned recv_scale), one kernel does it
+ * all: every CTA works out, from all the ids, the layout entries of the
+ * tokens it dispatches (one token per CTA when T + 1 CTAs fit on the GPU
+ * at once), with no CTA waiting on another; otherwise the call enqueues
+ * the two kernels of ep_get_layout and ep_dispatch (ep_kernel_launches
+ * tells which ran).
  *
  * idx .. recv_src, ws, ws_bytes: as ep_get_layout (ws is needed only when
  * ep_layout_workspace_bytes(T, k, E, R) > 0, i.e. for T*k > 2^19).
