@@ -3,19 +3,24 @@
 // every w[t,j] = 1 when no weights are given (a plain sum, as combining
 // per-rank partial outputs needs).
 //
-// Two kernels, both fp32 fma chains in slot order (so both bit-identical):
+// All kernels here run the same fp32 fma chain in slot order, so their
+// results are bit-identical to one another:
 //
-//  * combine_bulk_kernel (k <= 8, the common case): a bulk-copy (TMA)
-//    pipeline.  A CTA of kChunkVec threads walks a contiguous range of
-//    work items (token t, chunk c of kChunkVec 16-byte vectors).  Thread 0
-//    gathers the chunk of each of the token's k slot rows into shared
-//    memory with cp.async.bulk (one copy per row, completing on the stage's
-//    mbarrier), kStages items ahead; every thread then folds its 16 bytes
-//    of the k rows and writes one 16-byte vector of the output.  The bytes
-//    in flight live in shared memory, not registers, which is what keeps
-//    HBM busy on this read-dominated gather.
+//  * combine_bulk_kernel<chunk> (k <= 8, the common case): a bulk-copy
+//    (TMA) pipeline.  A CTA of `chunk` threads walks a contiguous range of
+//    work items (token t, chunk c of 16-byte vectors), the ranges of all
+//    CTAs equal to within one item.  Lanes 0..k-1 of warp 0 read the
+//    token's slot rows and weights and each gathers its row's chunk into
+//    shared memory with cp.async.bulk (completing on the stage's mbarrier),
+//    kStages items ahead; every thread then folds its 16 bytes of the k
+//    rows and writes one 16-byte vector of the output.  The bytes in flight
+//    live in shared memory, not registers, which keeps HBM busy on this
+//    read-dominated gather.  Chunks of 256 vectors, or 128 when each item
+//    then still gets a CTA of its own in one wave (small batches).
 //  * combine_reg_kernel (any k <= 32): a warp per item with 128-bit loads
 //    of 8 slot rows at a time into registers.
+//  * combine_fp8_bulk_kernel / combine_fp8_reg_kernel: the same for expert
+//    outputs kept as e4m3 codes plus block scales (below).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -29,9 +34,14 @@ namespace {
 constexpr int kRegThreads = 256;
 constexpr int kSlotBatch = 8;    // slot rows loaded together (register path)
 constexpr int kBulkMaxK = 8;     // slot rows one bulk stage holds
-constexpr int kChunkVec = 256;   // 16-byte vectors per row chunk = threads
 constexpr int kStages = 2;       // items in flight per CTA
-constexpr int kBulkSmem = kStages * kBulkMaxK * kChunkVec * 16;
+// 16-byte vectors per row chunk (= threads of the bulk kernel): 256 in
+// general; 128 when every item of the smaller chunks still gets a CTA of
+// its own in one wave (a decode batch), which shortens each CTA's chain.
+constexpr int kChunkVec = 256;
+constexpr int kSmallChunkVec = 128;
+template <int CHV>
+constexpr int bulk_smem() { return kStages * kBulkMaxK * CHV * 16; }
 
 __device__ __forceinline__ void fma_bf16x8(float *acc, float w, uint4 v) {
   const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -52,6 +62,7 @@ __device__ __forceinline__ uint4 to_bf16x8(const float *acc) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+template <int kChunkVec>
 __global__ void __launch_bounds__(kChunkVec)
     combine_bulk_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
                         const int32_t *__restrict__ slot_pos, const float *__restrict__ w,
@@ -394,19 +405,31 @@ cudaError_t launch_combine(const void *y, long n_rows, int T, int H, int k,
                            int32_t *d_err, cudaStream_t s, int *launches) {
   const int Hv = H / 8;
   if (k <= kBulkMaxK) {
-    const long items = static_cast<long>(T) * ((Hv + kChunkVec - 1) / kChunkVec);
-    if (items == 0) return cudaSuccess;
-    const cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(combine_bulk_kernel),
-                                               kBulkSmem);
+    auto launch = [&](auto kern, int chv, long items, long grid) -> cudaError_t {
+      ++*launches;
+      return launch_pdl(kern, dim3(grid), dim3(chv), chv * kStages * kBulkMaxK * 16, s, 1,
+                        static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,
+                        static_cast<uint4 *>(out), n_rows, d_err);
+    };
+    // small chunks when each of their items gets a CTA in one wave
+    {
+      auto kern = combine_bulk_kernel<kSmallChunkVec>;
+      constexpr int smem = bulk_smem<kSmallChunkVec>();
+      const long items = static_cast<long>(T) * ((Hv + kSmallChunkVec - 1) / kSmallChunkVec);
+      if (items == 0) return cudaSuccess;
+      const long cap = persistent_grid(reinterpret_cast<const void *>(kern), kSmallChunkVec,
+                                       smem, 1L << 40, num_sms);
+      if (items <= cap) return launch(kern, kSmallChunkVec, items, items);
+    }
+    auto kern = combine_bulk_kernel<kChunkVec>;
+    constexpr int smem = bulk_smem<kChunkVec>();
+    const cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
     if (err != cudaSuccess) return err;
+    const long items = static_cast<long>(T) * ((Hv + kChunkVec - 1) / kChunkVec);
     // CTAs: one per item, capped at the CTAs that fit on the SMs at once
-    const long grid = persistent_grid(reinterpret_cast<const void *>(combine_bulk_kernel),
-                                      kChunkVec, kBulkSmem, items * (kChunkVec / kWarp),
-                                      num_sms);
-    ++*launches;
-    return launch_pdl(combine_bulk_kernel, dim3(grid), dim3(kChunkVec), kBulkSmem, s, 1,
-                      static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,
-                      static_cast<uint4 *>(out), n_rows, d_err);
+    const long grid = persistent_grid(reinterpret_cast<const void *>(kern), kChunkVec, smem,
+                                      items * (kChunkVec / kWarp), num_sms);
+    return launch(kern, kChunkVec, items, grid);
   }
   const long items = static_cast<long>(T) * ((Hv + 31) / 32);
   if (items == 0) return cudaSuccess;
