@@ -44,6 +44,9 @@ __global__ void __launch_bounds__(kFp8BulkThreads)
   const long first = min(static_cast<long>(T), static_cast<long>(blockIdx.x) * per_cta);
   const long n_mine = min(static_cast<long>(T), first + per_cta) - first;
 
+  // the receive rows are written once and read by a later kernel: evict
+  // them first (measured: the step 0.3-0.5 % faster, the kernel ~1 %)
+  const uint64_t pol = l2_policy_evict_first();
   pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < kFp8BulkStages; ++s) mbar_init(&full[s], 1);
@@ -93,8 +96,8 @@ __global__ void __launch_bounds__(kFp8BulkThreads)
       for (int j = 0; j < k; ++j) {
         const int row = rows[i & 1][j];
         if (row < 0 || row >= n_rows) continue;
-        bulk_store(recv_q + static_cast<long>(row) * H, out_q, q_bytes);
-        bulk_store(recv_scale + static_cast<long>(row) * nb, out_s, s_bytes);
+        bulk_store(recv_q + static_cast<long>(row) * H, out_q, q_bytes, pol);
+        bulk_store(recv_scale + static_cast<long>(row) * nb, out_s, s_bytes, pol);
       }
       bulk_commit();
     }
