@@ -16,7 +16,11 @@ Prints one JSON line.  ``value`` is algorithmic HBM bytes moved per second
 over all ranks (each source byte read once, each destination byte written
 once); ``roofline`` is the dominant kernel against the measured copy
 bandwidth; ``decode`` is the 128-token decode workload in microseconds per
-call (layout + FP8 dispatch + combine), plain and in a CUDA graph;
+call (layout + FP8 dispatch + combine), unfused and with the fused
+layout + dispatch kernel, plain and in CUDA graphs; ``rank_dedup``,
+``combine_variants`` (aligned layout, FP8 combine, expert replicas) and
+``sm_budget_overlap`` (copy kernels beside a GEMM, with and without a
+green-context SM partition) measure the further forms of the path;
 ``cpu_baseline`` times the CPU oracle on a bounded sample; ``e2e`` runs the
 same step from pinned host buffers with the copies inside the timed region.
 
