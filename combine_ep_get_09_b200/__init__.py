@@ -42,6 +42,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep.so")
 
 _lib = None
 
+# e4m3 buffers may be given as torch's float8 type or as their raw bytes
+E4M3_BYTES = (torch.float8_e4m3fn, torch.uint8)
+
 
 class EPError(RuntimeError):
     def __init__(self, status: int, msg: str):
@@ -121,6 +124,43 @@ def _need_cuda(name: str, t: torch.Tensor):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _need(name: str, t: Optional[torch.Tensor], dtype, shape=None, min_rows=None):
+    """A CUDA, contiguous tensor of `dtype` and `shape` (or, with min_rows,
+    at least that many rows of shape[1:]): the library writes through the
+    raw pointer, so a wrong size would write out of bounds."""
+    if t is None:
+        raise ValueError(f"{name} is missing")
+    _need_cuda(name, t)
+    allowed = dtype if isinstance(dtype, tuple) else (dtype,)
+    if t.dtype not in allowed:
+        raise ValueError(f"{name} must be {' or '.join(map(str, allowed))}, not {t.dtype}")
+    if shape is not None:
+        if min_rows is not None:
+            if t.dim() != len(shape) or t.shape[0] < min_rows or tuple(t.shape[1:]) != tuple(shape[1:]):
+                raise ValueError(f"{name} must have shape [>= {min_rows}, "
+                                 f"{', '.join(map(str, shape[1:]))}], not {tuple(t.shape)}")
+        elif tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+
+
+def _need_err(d_err: Optional[torch.Tensor]):
+    if d_err is not None:
+        _need("d_err", d_err, torch.int32)
+        if d_err.numel() < 1:
+            raise ValueError("d_err needs one element")
+
+
+def _check_layout(L, T: int, k: int, E: int, R: int):
+    i32 = torch.int32
+    _need("cnt_e", L.cnt_e, i32, (E,))
+    _need("cnt_r", L.cnt_r, i32, (R,))
+    _need("in_rank", L.in_rank, torch.uint8, (T, R))
+    _need("off_e", L.off_e, i32, (E + 1,))
+    _need("off_r", L.off_r, i32, (R + 1,))
+    _need("slot_pos", L.slot_pos, i32, (T, k))
+    _need("recv_src", L.recv_src, i32, (T * k,))
+
+
 class Layout(NamedTuple):
     cnt_e: torch.Tensor     # [E] int32
     cnt_r: torch.Tensor     # [R] int32
@@ -161,6 +201,8 @@ def ep_get_layout(idx: torch.Tensor, E: int, R: int, *,
     T, k = idx.shape
     if out is None:
         out = empty_layout(T, k, E, R, idx.device)
+    _check_layout(out, T, k, E, R)
+    _need_err(d_err)
     need = ep_layout_workspace_bytes(T, k, E, R)
     if ws is None and need > 0:
         ws = torch.zeros(need, dtype=torch.uint8, device=idx.device)
@@ -189,6 +231,8 @@ def ep_get_layout_noalloc(idx: torch.Tensor, E: int, R: int, *,
     T, k = idx.shape
     if out is None:
         out = empty_layout(T, k, E, R, idx.device)
+    _check_layout(out, T, k, E, R)
+    _need_err(d_err)
     _check(lib().ep_get_layout_noalloc(
         _ptr(idx), int(idx.dtype == torch.int64), T, k, E, R,
         _ptr(out.cnt_e), _ptr(out.cnt_r), _ptr(out.in_rank), _ptr(out.off_e),
@@ -223,6 +267,10 @@ def ep_get_rank_layout(in_rank: torch.Tensor, *, out: Optional[RankLayout] = Non
         i32 = dict(dtype=torch.int32, device=dev)
         out = RankLayout(torch.empty(R, **i32), torch.empty(R + 1, **i32),
                          torch.empty((T, R), **i32), torch.empty(T * R, **i32))
+    _need("cnt_r", out.cnt_r, torch.int32, (R,))
+    _need("off_r", out.off_r, torch.int32, (R + 1,))
+    _need("rank_row", out.rank_row, torch.int32, (T, R))
+    _need("rank_src", out.rank_src, torch.int32, (T * R,))
     need = ep_rank_layout_workspace_bytes(T, R)
     if ws is None and need > 0:
         ws = torch.zeros(need, dtype=torch.uint8, device=dev)
@@ -247,17 +295,21 @@ def ep_dispatch(x: torch.Tensor, slot_pos: torch.Tensor, fp8: bool = False, *,
     if x.dtype != torch.bfloat16 or slot_pos.dtype != torch.int32:
         raise ValueError("x must be bf16 and slot_pos int32")
     T, H = x.shape
+    if slot_pos.dim() != 2 or slot_pos.shape[0] != T:
+        raise ValueError("slot_pos must be [T, k] with x's T")
     k = slot_pos.shape[1]
+    rdt = torch.float8_e4m3fn if fp8 else torch.bfloat16
     if recv is None:
-        recv = torch.empty((T * k, H), device=x.device,
-                           dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16)
-    if fp8 and recv_scale is None:
-        recv_scale = torch.empty((recv.shape[0], H // 128), device=x.device,
-                                 dtype=torch.float32)
-    if fp8 and recv_scale.shape[0] < recv.shape[0]:
-        raise ValueError("recv_scale needs a row per receive row")
+        recv = torch.empty((T * k, H), device=x.device, dtype=rdt)
+    _need("recv", recv, E4M3_BYTES if fp8 else rdt, (0, H), min_rows=0)
+    if fp8:
+        if recv_scale is None:
+            recv_scale = torch.empty((recv.shape[0], H // 128), device=x.device,
+                                     dtype=torch.float32)
+        _need("recv_scale", recv_scale, torch.float32, (0, H // 128), min_rows=recv.shape[0])
     if recv.shape[0] == 0 and T * k > 0:
         raise ValueError("recv has no rows")   # 0 would mean T*k rows to the library
+    _need_err(d_err)
     _check(lib().ep_dispatch(_ptr(x), T, H, k, _ptr(slot_pos), int(bool(fp8)),
                              _ptr(recv), _ptr(recv_scale) if fp8 else None,
                              recv.shape[0], num_sms, _ptr(d_err), _stream(stream)))
@@ -283,11 +335,16 @@ def ep_layout_dispatch(idx: torch.Tensor, E: int, R: int, x: torch.Tensor,
     H = x.shape[1]
     if out is None:
         out = empty_layout(T, k, E, R, idx.device)
+    _check_layout(out, T, k, E, R)
+    rdt = torch.float8_e4m3fn if fp8 else torch.bfloat16
     if recv is None:
-        recv = torch.empty((T * k, H), device=x.device,
-                           dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16)
-    if fp8 and recv_scale is None:
-        recv_scale = torch.empty((T * k, H // 128), device=x.device, dtype=torch.float32)
+        recv = torch.empty((T * k, H), device=x.device, dtype=rdt)
+    _need("recv", recv, E4M3_BYTES if fp8 else rdt, (T * k, H), min_rows=T * k)
+    if fp8:
+        if recv_scale is None:
+            recv_scale = torch.empty((T * k, H // 128), device=x.device, dtype=torch.float32)
+        _need("recv_scale", recv_scale, torch.float32, (T * k, H // 128), min_rows=T * k)
+    _need_err(d_err)
     need = ep_layout_workspace_bytes(T, k, E, R)
     if ws is None and need > 0:
         ws = torch.zeros(need, dtype=torch.uint8, device=idx.device)
@@ -316,8 +373,12 @@ def ep_combine(y: torch.Tensor, slot_pos: torch.Tensor, w: Optional[torch.Tensor
         raise ValueError("y must be bf16 and w fp32")
     T, k = slot_pos.shape
     H = y.shape[1]
+    if w is not None and tuple(w.shape) != (T, k):
+        raise ValueError(f"w must have shape {(T, k)}")
     if out is None:
         out = torch.empty((T, H), device=y.device, dtype=torch.bfloat16)
+    _need("out", out, torch.bfloat16, (T, H))
+    _need_err(d_err)
     if y.shape[0] == 0 and T > 0:
         raise ValueError("y has no rows")   # 0 would mean T*k rows to the library
     _check(lib().ep_combine(_ptr(y), y.shape[0], T, H, k, _ptr(slot_pos), _ptr(w),
@@ -337,14 +398,18 @@ def ep_combine_fp8(y_q: torch.Tensor, y_scale: torch.Tensor, slot_pos: torch.Ten
         _need_cuda(name, t)
     if w is not None:
         _need_cuda("w", w)
-    if y_q.dtype != torch.float8_e4m3fn or y_scale.dtype != torch.float32:
-        raise ValueError("y_q must be float8_e4m3fn and y_scale fp32")
+    if y_q.dtype not in E4M3_BYTES or y_scale.dtype != torch.float32:
+        raise ValueError("y_q must be float8_e4m3fn (or its uint8 bytes) and y_scale fp32")
     T, k = slot_pos.shape
     rows, H = y_q.shape
     if (rows == 0 and T > 0) or y_scale.shape != (rows, H // 128):
         raise ValueError("y_scale must be [rows, H/128] and y_q hold rows")
+    if w is not None and tuple(w.shape) != (T, k):
+        raise ValueError(f"w must have shape {(T, k)}")
     if out is None:
         out = torch.empty((T, H), device=y_q.device, dtype=torch.bfloat16)
+    _need("out", out, torch.bfloat16, (T, H))
+    _need_err(d_err)
     _check(lib().ep_combine_fp8(_ptr(y_q), _ptr(y_scale), rows, T, H, k, _ptr(slot_pos),
                                 _ptr(w), _ptr(out), num_sms, _ptr(d_err), _stream(stream)))
     return out
@@ -373,6 +438,10 @@ def ep_pad_layout(layout: Layout, align: int, *, out: Optional[PaddedLayout] = N
         i32 = dict(dtype=torch.int32, device=dev)
         out = PaddedLayout(torch.empty(E + 1, **i32), torch.empty((T, k), **i32),
                            torch.empty(max(1, ep_aligned_rows(T, k, E, align)), **i32))
+    _need("off_pad", out.off_pad, torch.int32, (E + 1,))
+    _need("slot_pos", out.slot_pos, torch.int32, (T, k))
+    _need("recv_src", out.recv_src, torch.int32, (0,),
+          min_rows=ep_aligned_rows(T, k, E, align))
     _check(lib().ep_pad_layout(_ptr(layout.cnt_e), _ptr(layout.slot_pos), T, k, E, align,
                                _ptr(out.off_pad), _ptr(out.slot_pos), _ptr(out.recv_src),
                                _stream(stream)))
@@ -403,6 +472,8 @@ def ep_map_replicas(idx: torch.Tensor, layout: Layout, rep_off: torch.Tensor,
         raise ValueError("rep_off needs E + 1 entries for the layout's E experts")
     if out is None:
         out = torch.empty((T, k), dtype=torch.int32, device=idx.device)
+    _need("out", out, torch.int32, (T, k))
+    _need_err(d_err)
     _check(lib().ep_map_replicas(_ptr(idx), int(idx.dtype == torch.int64), T, k, E,
                                  _ptr(layout.slot_pos), _ptr(layout.off_e), _ptr(rep_off),
                                  _ptr(rep_ids), _ptr(out), _ptr(d_err), _stream(stream)))
