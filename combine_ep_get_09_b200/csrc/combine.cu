@@ -15,7 +15,7 @@
 //    kStages items ahead; every thread then folds its 16 bytes of the k
 //    rows and writes one 16-byte vector of the output.  The bytes in flight
 //    live in shared memory, not registers, which keeps HBM busy on this
-//    read-dominated gather.  Chunks of 256 vectors, or 128 when each item
+//    read-dominated gather.  Chunks of 256 vectors, or 64 when each item
 //    then still gets a CTA of its own in one wave (small batches).
 //  * combine_reg_kernel (any k <= 32): a warp per item with 128-bit loads
 //    of 8 slot rows at a time into registers.
@@ -36,10 +36,11 @@ constexpr int kSlotBatch = 8;    // slot rows loaded together (register path)
 constexpr int kBulkMaxK = 8;     // slot rows one bulk stage holds
 constexpr int kStages = 2;       // items in flight per CTA
 // 16-byte vectors per row chunk (= threads of the bulk kernel): 256 in
-// general; 128 when every item of the smaller chunks still gets a CTA of
-// its own in one wave (a decode batch), which shortens each CTA's chain.
+// general; 64 when every item of the smaller chunks still gets a CTA of its
+// own in one wave (a decode batch), which shortens each CTA's chain.  (128
+// fits one wave only where 64 does too: 6 of its CTAs fit an SM, 13 of 64's.)
 constexpr int kChunkVec = 256;
-constexpr int kSmallChunkVec = 128;
+constexpr int kSmallChunkVec = 64;
 template <int CHV>
 constexpr int bulk_smem() { return kStages * kBulkMaxK * CHV * 16; }
 
@@ -414,14 +415,12 @@ cudaError_t launch_combine(const void *y, long n_rows, int T, int H, int k,
                         static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,
                         static_cast<uint4 *>(out), n_rows, d_err);
     };
-    // small chunks when each of their items gets a CTA in one wave
-    {
+    if (T == 0) return cudaSuccess;
+    {  // small chunks when each of their items gets a CTA in one wave
       auto kern = combine_bulk_kernel<kSmallChunkVec>;
-      constexpr int smem = bulk_smem<kSmallChunkVec>();
       const long items = static_cast<long>(T) * ((Hv + kSmallChunkVec - 1) / kSmallChunkVec);
-      if (items == 0) return cudaSuccess;
       const long cap = persistent_grid(reinterpret_cast<const void *>(kern), kSmallChunkVec,
-                                       smem, 1L << 40, num_sms);
+                                       bulk_smem<kSmallChunkVec>(), 1L << 40, num_sms);
       if (items <= cap) return launch(kern, kSmallChunkVec, items, items);
     }
     auto kern = combine_bulk_kernel<kChunkVec>;
