@@ -355,6 +355,8 @@ def bench_ours(args, world, rank, device):
         result["decode"] = bench_decode(ep, device, world)
     if not args.skip_dedup:
         result["rank_dedup"] = bench_rank_dedup(ep, st, cfg, device, world)
+    if not args.skip_workloads:
+        result["other_workloads"] = bench_workloads(ep, device, world)
     if not args.skip_variants:
         result["combine_variants"] = bench_combine_variants(ep, st, cfg, device, world)
         result["combine_variants"]["replicas"] = bench_replicas(ep, device, world)
@@ -468,6 +470,46 @@ def bench_rank_dedup(ep, st, cfg, device, world, iters=20):
                             world, device)
         res[name] = {"us": round(us, 2), "bytes": nbytes,
                      "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)}
+    return res
+
+
+def bench_workloads(ep, device, world, names=("skewed", "large"), iters=10):
+    """The step's kernels on the other full-size shapes, each step after an
+    L2 flush, timed with CUDA events around each kernel (like the prefill
+    step): the skewed batch (Zipf-popular experts, 8192 tokens) and the large
+    one (32768 tokens of H=4096 over 128 experts in 16 ranks)."""
+    res = {}
+    for name in names:
+        cfg = workloads.CONFIGS[name]
+        st = Step(ep, cfg, workloads.make_batch(cfg, seed=0), device)
+        stream = torch.cuda.Stream(device)
+        flush = L2Flush(device)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(iters)]
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                flush()
+                st.run(stream)
+            for e in evs:
+                flush()
+                st.run(stream, e)
+        stream.synchronize()
+        if ep.ep_read_error(st.d_err, stream) != 0:
+            raise RuntimeError(f"the device reported an error on the {name} workload")
+        nbytes = step_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R)
+        out = {"T": cfg.T, "H": cfg.H, "E": cfg.E, "R": cfg.R, "k": cfg.k}
+        for j, n in enumerate(KERNELS):
+            us = max_over_ranks(statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) * 1e3,
+                                world, device)
+            gbs = nbytes[n] / (us * 1e-6) / 1e9
+            out[n] = {"us": round(us, 2), "bytes": nbytes[n], "GB/s": round(gbs, 1),
+                      "frac_of_8TBs": round(gbs / SPEC_HBM_GBS, 4)}
+        step_us = max_over_ranks(statistics.mean(e[0].elapsed_time(e[4]) for e in evs) * 1e3,
+                                 world, device)
+        out["step_us"] = round(step_us, 2)
+        out["step_GB/s"] = round(sum(nbytes.values()) / (step_us * 1e-6) / 1e9, 1)
+        res[name] = out
+        del st
+        torch.cuda.empty_cache()
     return res
 
 
@@ -977,11 +1019,55 @@ def cpu_baseline(cfg, batch, seconds: float, sample_tokens: int = 512):
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return {"value": round(nb * reps / el / 1e9, 3), "unit": "GB/s", "cores": 1,
+    res = {"value": round(nb * reps / el / 1e9, 3), "unit": "GB/s", "cores": 1,
+           "kind": "oracle",
+           "sample": (f"first {sample_tokens} tokens of the prefill batch, whole step "
+                      f"(layout + bf16 dispatch + FP8 dispatch + combine), "
+                      f"{reps} reps in {el:.1f} s, single-threaded C oracle")}
+    res["all_cores"] = cpu_baseline_threads(cfg, batch, seconds, sample_tokens, nb)
+    return res
+
+
+def cpu_baseline_threads(cfg, batch, seconds: float, sample_tokens: int, nb: int,
+                         max_threads: int = 64):
+    """The same oracle step on every host core at once: one Python thread per
+    core (the C oracle runs without the interpreter lock), each on its own
+    `sample_tokens`-token slice of the batch, for about `seconds`."""
+    import threading
+    import oracle
+    n = max(1, min(len(os.sched_getaffinity(0)), max_threads))
+    n_slices = max(1, batch.x.shape[0] // sample_tokens)
+    slices = []
+    for i in range(min(n, n_slices)):
+        a = i * sample_tokens
+        slices.append(tuple(t[a:a + sample_tokens].contiguous()
+                            for t in (batch.x, batch.idx, batch.w)))
+    reps = [0] * n
+    start = threading.Barrier(n + 1)
+    stop = time.perf_counter() + 1e9
+
+    def work(i):
+        x, idx, w = slices[i % len(slices)]
+        start.wait()
+        while time.perf_counter() < stop:
+            oracle_sample_step(oracle, cfg, x, idx, w)
+            reps[i] += 1
+
+    threads = [threading.Thread(target=work, args=(i,), daemon=True) for i in range(n)]
+    for t in threads:
+        t.start()
+    t0 = time.perf_counter()
+    stop = t0 + seconds
+    start.wait()
+    for t in threads:
+        t.join()
+    el = time.perf_counter() - t0
+    total = sum(reps)
+    return {"value": round(nb * total / el / 1e9, 3), "unit": "GB/s", "cores": n,
             "kind": "oracle",
-            "sample": (f"first {sample_tokens} tokens of the prefill batch, whole step "
-                       f"(layout + bf16 dispatch + FP8 dispatch + combine), "
-                       f"{reps} reps in {el:.1f} s, single-threaded C oracle")}
+            "sample": (f"{n} threads, each repeating the step on one of {len(slices)} "
+                       f"{sample_tokens}-token slices of the prefill batch; "
+                       f"{total} steps in {el:.1f} s")}
 
 
 def bench_reference(args, world, rank):
@@ -1082,6 +1168,8 @@ def main():
     p.add_argument("--skip-dedup", action="store_true")
     p.add_argument("--skip-overlap", action="store_true")
     p.add_argument("--skip-variants", action="store_true")
+    p.add_argument("--skip-workloads", action="store_true",
+                   help="skip the skewed and large shapes")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--reference-tokens", type=int, default=256)
     p.add_argument("--profile", choices=("layout", "dispatch_bf16", "dispatch_fp8", "combine",
