@@ -296,6 +296,8 @@ def bench_ours(args, world, rank, device):
     launches = ep.ep_kernel_launches() - launches0
     if ep.ep_read_error(st.d_err, stream) != 0:
         raise RuntimeError("the device reported an error in the timed steps")
+    back_to_back = bench_back_to_back(st, stream, flush, args.steps, world, device,
+                                      total_bytes)
 
     per_kernel = {n: [] for n in KERNELS}
     step_ms = []
@@ -350,6 +352,7 @@ def bench_ours(args, world, rank, device):
                      "algorithmic_bytes": nbytes[dom]},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
+        "back_to_back": back_to_back,
     }
     if not args.skip_decode:
         result["decode"] = bench_decode(ep, device, world)
@@ -471,6 +474,30 @@ def bench_rank_dedup(ep, st, cfg, device, world, iters=20):
         res[name] = {"us": round(us, 2), "bytes": nbytes,
                      "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)}
     return res
+
+
+def bench_back_to_back(st, stream, flush, steps, world, device, total_bytes):
+    """The same steps with events only at their start and end, after the
+    timed region: the four kernels then run back to back as a caller issues
+    them, each launched as the previous one's last CTAs exit (an event
+    recorded between two kernels makes the second wait for the event)."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            flush()
+            a.record(stream)
+            st.run(stream)
+            b.record(stream)
+        stream.synchronize()
+    barrier(world)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, device)
+    return {"value": round(job_value(total_bytes, steps, world, ms), 1), "unit": "GB/s",
+            "us_per_step": round(ms / steps * 1e3, 2), "steps": steps,
+            "how": "events at each step's start and end only; the same L2 flush "
+                   "between steps"}
 
 
 def bench_workloads(ep, device, world, names=("skewed", "large"), iters=10):

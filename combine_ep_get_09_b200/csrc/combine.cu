@@ -82,7 +82,6 @@ __global__ void __launch_bounds__(kChunkVec)
   const long first = items * blockIdx.x / gridDim.x;
   const long n_mine = items * (blockIdx.x + 1) / gridDim.x - first;
 
-  pdl_trigger();
   if (tid == 0) {
     // every lane of warp 0 arrives once per phase (see issue)
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], kWarp);
@@ -159,7 +158,6 @@ __global__ void __launch_bounds__(kRegThreads, 2)
     combine_reg_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
                        const int32_t *__restrict__ slot_pos, const float *__restrict__ w,
                        uint4 *__restrict__ out, long n_rows) {
-  pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int nchunks = (Hv + 31) / 32;
@@ -268,7 +266,6 @@ __global__ void __launch_bounds__(kQChunkVec)
            j * (kQChunkVec / 8);
   };
 
-  pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], kWarp);
     mbar_init_fence();
@@ -345,7 +342,6 @@ __global__ void __launch_bounds__(kRegThreads, 2)
                            int T, int H, int k, const int32_t *__restrict__ slot_pos,
                            const float *__restrict__ w, uint4 *__restrict__ out,
                            long n_rows) {
-  pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int Hq = H >> 4, nb = H >> 7;

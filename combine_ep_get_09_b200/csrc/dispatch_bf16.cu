@@ -5,7 +5,8 @@
 // loads, then writes it to each of the token's k receive rows with
 // coalesced streaming stores, so HBM sees each source byte read once and
 // each destination byte written once.  The slot rows of the token are
-// fetched by lanes 0..k-1 and broadcast with shuffles.
+// fetched by lanes 0..k-1 and broadcast with shuffles.  Before waiting on
+// the previous kernel, every warp asks L2 for the x chunks it will copy.
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -13,19 +14,40 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kBf16Vec = 2;  // 16-byte vectors per lane per item
+// x bytes the kernel prefetches into L2 before its wait (half of the 126 MB
+// L2: the whole token batch at the prefill shape; the first part of larger
+// ones, which prefetching entirely slowed by 5 % as lines were evicted
+// before their turn)
+constexpr long kPrefetchBytes = 64L << 20;
 
+// 8 CTAs per SM (at most 32 registers; the uncapped build took 36 and left
+// room for 6): measured 0.7 us faster at the prefill shape.
 template <int V>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 8)
     dispatch_bf16_kernel(const uint4 *__restrict__ x, int T, int Hv, int k,
                          const int32_t *__restrict__ slot_pos,
                          uint4 *__restrict__ recv, long n_rows) {
-  pdl_trigger();
-  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int per_chunk = 32 * V;
   const int nchunks = (Hv + per_chunk - 1) / per_chunk;
   const long items = static_cast<long>(T) * nchunks;
   const long nwarps = (static_cast<long>(gridDim.x) * blockDim.x) >> 5;
+  {
+    // ask L2 for this warp's first x chunks up front, one bulk prefetch per
+    // lane and item, before waiting on the previous kernel (a prefetch only
+    // warms L2, which every later write goes through, so it is safe even
+    // when that kernel writes x).  Only the items of the first
+    // kPrefetchBytes of x in loop order: more would be evicted before use.
+    const long w0 = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const long pf_end = min(items, kPrefetchBytes / (per_chunk * 16));
+    for (long it = w0 + static_cast<long>(lane) * nwarps; it < pf_end; it += 32 * nwarps) {
+      const int t = static_cast<int>(it / nchunks);
+      const int c = static_cast<int>(it - static_cast<long>(t) * nchunks);
+      prefetch_l2(x + static_cast<long>(t) * Hv + c * per_chunk,
+                  min(per_chunk, Hv - c * per_chunk) * 16);
+    }
+  }
+  pdl_wait();
   for (long it = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
        it < items; it += nwarps) {
     const int t = static_cast<int>(it / nchunks);

@@ -47,7 +47,6 @@ __global__ void __launch_bounds__(kFp8BulkThreads)
   // the receive rows are written once and read by a later kernel: evict
   // them first (measured: the step 0.3-0.5 % faster, the kernel ~1 %)
   const uint64_t pol = l2_policy_evict_first();
-  pdl_trigger();
   if (tid == 0) {
     for (int s = 0; s < kFp8BulkStages; ++s) mbar_init(&full[s], 1);
     mbar_init_fence();
@@ -122,7 +121,6 @@ __global__ void __launch_bounds__(kThreads)
                         const int32_t *__restrict__ slot_pos,
                         uint2 *__restrict__ recv_q,
                         float *__restrict__ recv_scale, long n_rows) {
-  pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31, half = lane >> 4, sub = lane & 15;
   const int Hv = H >> 3;   // 8-channel units per row (16 B in, 8 B out)

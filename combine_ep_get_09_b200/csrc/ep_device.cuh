@@ -43,16 +43,22 @@ __device__ __forceinline__ void st_stream_f32(float *p, float v) {
 
 // Programmatic dependent launch (sm_90+).  Every kernel of the library is
 // launched with programmatic stream serialization, so it may be scheduled
-// while the previous kernel on the stream is still running; it must call
+// while the previous kernel on the stream is still finishing; it must call
 // pdl_wait() before touching memory that kernel writes (griddepcontrol.wait
 // returns once the previous grid has completed and its writes are visible;
-// with no such predecessor it returns at once).  pdl_trigger() lets the
-// next kernel on the stream be scheduled early; that kernel still waits for
-// this one to finish before using its output.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+// with no such predecessor it returns at once).  No kernel issues
+// griddepcontrol.launch_dependents: a CTA's exit counts as its trigger, so
+// the next kernel is launched as this one's last CTAs leave, which hides
+// its launch latency without parking its CTAs on SMs that are still busy.
+// (Triggering at kernel entry measured slower everywhere: 288 vs 256 us
+// for a back-to-back prefill step, 8.23 vs 8.12 us for a decode call.)
+// Bulk prefetch of [p, p + bytes) into L2 (p 16-byte aligned, bytes a
+// multiple of 16); a hint with no completion to wait for.
+__device__ __forceinline__ void prefetch_l2(const void *p, int bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;

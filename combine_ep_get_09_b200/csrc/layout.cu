@@ -381,7 +381,6 @@ __device__ int scan_counts(int *a, int n, int32_t *cnt, int32_t *off) {
 
 template <typename IdT>
 __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Params p) {
-  pdl_trigger();
   cg::cluster_group cluster = cg::this_cluster();
   const int n_ctas = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
@@ -472,7 +471,6 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
 
 template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
-  pdl_trigger();
   pdl_wait();
   extern __shared__ int smem[];
   const int E = p.E, R = p.R, C = E + R, ld = hist_ld(p);
@@ -583,7 +581,6 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
 
 template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads) layout_place_kernel(Params p) {
-  pdl_trigger();
   pdl_wait();
   extern __shared__ int smem[];
   const int E = p.E, C = p.E + p.R, ld = hist_ld(p);

@@ -177,7 +177,6 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(const FusedAr
   const int in_bytes = 2 * H;
   const bool lead = blockIdx.x == 0;
 
-  pdl_trigger();
   // thread 0: token first + i -> input stage i % kStages
   auto issue = [&](int i) {
     const int s = i % kStages;
@@ -460,7 +459,6 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
   const bool counts_cta = t == T;
   const IdT *idx = static_cast<const IdT *>(a.idx);
 
-  pdl_trigger();
   if (tid == 0 && !counts_cta) {
     mbar_init(&full, 1);
     mbar_init_fence();

@@ -42,7 +42,6 @@ __global__ void __launch_bounds__(kPadThreads)
   int *offp = off + E + 1;  // [E + 1] padded offsets
   const int tid = threadIdx.x, lane = tid & 31;
 
-  pdl_trigger();
   pdl_wait();
   for (int e = tid; e < E; e += kPadThreads) cnt[e] = __ldg(cnt_e + e);
   __syncthreads();

@@ -20,7 +20,6 @@ __global__ void __launch_bounds__(kRepThreads)
                         const int32_t *__restrict__ slot_pos, const int32_t *__restrict__ off_e,
                         const int32_t *__restrict__ rep_off, const int32_t *__restrict__ rep_ids,
                         int32_t *__restrict__ phys, int32_t *d_err) {
-  pdl_trigger();
   pdl_wait();
   for (long i = static_cast<long>(blockIdx.x) * kRepThreads + threadIdx.x; i < n;
        i += static_cast<long>(gridDim.x) * kRepThreads) {
