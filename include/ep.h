@@ -34,6 +34,12 @@
  *    EP_ERR_TIMEOUT if a kernel's bounded wait for its own asynchronous
  *    copies gave up (it then stops early instead of hanging).
  *  - Pointers must be 16-byte aligned unless stated otherwise.
+ *  - Kernels are launched with programmatic stream serialization: one may
+ *    be scheduled as the previous kernel on `stream` finishes, and it waits
+ *    for that kernel (griddepcontrol.wait) before reading anything.  None
+ *    releases its successor early.  A caller's kernel launched after one of
+ *    these with the same attribute must wait the same way before reading
+ *    their output; one launched without it sees plain stream order.
  */
 #ifndef EP_H_
 #define EP_H_
