@@ -64,6 +64,7 @@ _SIGNATURES = {
     "ep_abi_version": ([], _i),
     "ep_last_error_string": ([], ctypes.c_char_p),
     "ep_kernel_launches": ([], ctypes.c_uint64),
+    "ep_debug_expire_first_wait": ([_i], None),
     "ep_layout_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "ep_get_layout": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
                        _vp, _vp, _sz, _vp, _vp], _i),
@@ -179,6 +180,14 @@ def ep_kernel_launches() -> int:
     return int(lib().ep_kernel_launches())
 
 
+def ep_debug_expire_first_wait(on: bool) -> None:
+    """Testing switch: while on, the first bounded copy wait of every CTA of
+    the bulk-copy kernels gives up at once, so their time-out path
+    (EP_ERR_TIMEOUT in d_err, drain, early return) runs; off restores the
+    normal limit.  Process-wide."""
+    lib().ep_debug_expire_first_wait(1 if on else 0)
+
+
 def empty_layout(T: int, k: int, E: int, R: int, device) -> Layout:
     i32 = dict(dtype=torch.int32, device=device)
     return Layout(torch.empty(E, **i32), torch.empty(R, **i32),
@@ -221,11 +230,19 @@ def ep_get_layout_noalloc(idx: torch.Tensor, E: int, R: int, *,
                           stream=None) -> Layout:
     """ep_get_layout for callers that cannot allocate device memory: the
     library's fixed scratch array (EP_NOALLOC_SCRATCH_BYTES per device)
-    replaces the workspace.  Calls that overlap on the GPU race on that
-    array; the first call on a device looks its address up, so make it
-    before any stream capture.  Outputs are allocated here only when
-    ``out`` is not given."""
+    replaces the workspace.  The array used is the current device's, so
+    ``idx``, the outputs and ``stream`` must be on the current device.
+    Calls that overlap on the GPU race on that array; the first call on a
+    device loads the library's module there, so make it before any stream
+    capture.  Outputs are allocated here only when ``out`` is not given."""
     _need_cuda("idx", idx)
+    cur = torch.cuda.current_device()
+    if idx.device.index != cur:
+        raise ValueError(f"idx is on cuda:{idx.device.index} but the current device is "
+                         f"cuda:{cur}; the scratch array used is the current device's")
+    if isinstance(stream, torch.cuda.Stream) and stream.device.index != cur:
+        raise ValueError(f"stream belongs to cuda:{stream.device.index} but the current "
+                         f"device is cuda:{cur}")
     if idx.dtype not in (torch.int64, torch.int32) or idx.dim() != 2:
         raise ValueError("idx must be a 2-D int64 or int32 tensor")
     T, k = idx.shape

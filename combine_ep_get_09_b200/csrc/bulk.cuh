@@ -49,12 +49,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
 
 // Bounded wait for the phase of parity `parity` to complete.  Each try_wait
 // may suspend the thread for a short hardware-defined time; after
-// kMaxBarrierPolls unsuccessful tries the wait gives up and returns false,
-// so a copy that never lands cannot hang the GPU.
+// `max_polls` (normally kMaxBarrierPolls) unsuccessful tries the wait gives
+// up and returns false, so a copy that never lands cannot hang the GPU.
+// A kernel passes 0 for its first wait only when the library's testing
+// switch (ep_debug_expire_first_wait) is on: that wait then gives up
+// without polling while the copy still lands, which runs the kernel's
+// time-out path (report, drain, return) on demand.
 constexpr int kMaxBarrierPolls = 1 << 22;
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
-  for (int i = 0; i < kMaxBarrierPolls; ++i)
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity,
+                                                  int max_polls = kMaxBarrierPolls) {
+  for (int i = 0; i < max_polls; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }

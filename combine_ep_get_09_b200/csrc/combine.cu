@@ -34,12 +34,18 @@ namespace {
 constexpr int kRegThreads = 256;
 constexpr int kSlotBatch = 8;    // slot rows loaded together (register path)
 constexpr int kBulkMaxK = 8;     // slot rows one bulk stage holds
-constexpr int kStages = 2;       // items in flight per CTA
+#ifndef EP_COMBINE_STAGES
+#define EP_COMBINE_STAGES 2
+#endif
+#ifndef EP_COMBINE_CHV
+#define EP_COMBINE_CHV 256
+#endif
+constexpr int kStages = EP_COMBINE_STAGES;       // items in flight per CTA
 // 16-byte vectors per row chunk (= threads of the bulk kernel): 256 in
 // general; 64 when every item of the smaller chunks still gets a CTA of its
 // own in one wave (a decode batch), which shortens each CTA's chain.  (128
 // fits one wave only where 64 does too: 6 of its CTAs fit an SM, 13 of 64's.)
-constexpr int kChunkVec = 256;
+constexpr int kChunkVec = EP_COMBINE_CHV;
 constexpr int kSmallChunkVec = 64;
 template <int CHV>
 constexpr int bulk_smem() { return kStages * kBulkMaxK * CHV * 16; }
@@ -67,7 +73,8 @@ template <int kChunkVec>
 __global__ void __launch_bounds__(kChunkVec)
     combine_bulk_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
                         const int32_t *__restrict__ slot_pos, const float *__restrict__ w,
-                        uint4 *__restrict__ out, long n_rows, int32_t *d_err) {
+                        uint4 *__restrict__ out, long n_rows, int first_polls,
+                        int32_t *d_err) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   uint4 *stage_buf = reinterpret_cast<uint4 *>(smem_raw);  // [kStages][kBulkMaxK][kChunkVec]
   __shared__ __align__(8) uint64_t full[kStages];
@@ -128,7 +135,8 @@ __global__ void __launch_bounds__(kChunkVec)
     const long it = first + i;
     const int t = static_cast<int>(it / nchunks);
     const int v0 = static_cast<int>(it % nchunks) * kChunkVec;
-    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1));
+    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1),
+                                      i == 0 ? first_polls : kMaxBarrierPolls);
     if (__syncthreads_or(!ok)) {
       timed_out = true;
       break;
@@ -244,7 +252,7 @@ __global__ void __launch_bounds__(kQChunkVec)
     combine_fp8_bulk_kernel(const uint4 *__restrict__ y_q, const float *__restrict__ y_scale,
                             int T, int H, int k, const int32_t *__restrict__ slot_pos,
                             const float *__restrict__ w, uint4 *__restrict__ out, long n_rows,
-                            int32_t *d_err) {
+                            int first_polls, int32_t *d_err) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t full[kStages];
   __shared__ int stage_row[kStages][kBulkMaxK];
@@ -310,7 +318,8 @@ __global__ void __launch_bounds__(kQChunkVec)
     const long it = first + i;
     const int t = static_cast<int>(it / nchunks);
     const int v0 = static_cast<int>(it % nchunks) * kQChunkVec;
-    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1));
+    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kStages) & 1),
+                                      i == 0 ? first_polls : kMaxBarrierPolls);
     if (__syncthreads_or(!ok)) {
       timed_out = true;
       break;
@@ -388,7 +397,7 @@ cudaError_t launch_combine_fp8(const void *y_q, const float *y_scale, long n_row
     ++*launches;
     return launch_pdl(combine_fp8_bulk_kernel, dim3(grid), dim3(kQChunkVec), kQBulkSmem, s, 1,
                       static_cast<const uint4 *>(y_q), y_scale, T, H, k, slot_pos, w,
-                      static_cast<uint4 *>(out), n_rows, d_err);
+                      static_cast<uint4 *>(out), n_rows, first_wait_polls(), d_err);
   }
   const long items = static_cast<long>(T) * ((Hq + 31) / 32);
   if (items == 0) return cudaSuccess;
@@ -409,7 +418,7 @@ cudaError_t launch_combine(const void *y, long n_rows, int T, int H, int k,
       ++*launches;
       return launch_pdl(kern, dim3(grid), dim3(chv), chv * kStages * kBulkMaxK * 16, s, 1,
                         static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,
-                        static_cast<uint4 *>(out), n_rows, d_err);
+                        static_cast<uint4 *>(out), n_rows, first_wait_polls(), d_err);
     };
     if (T == 0) return cudaSuccess;
     {  // small chunks when each of their items gets a CTA in one wave

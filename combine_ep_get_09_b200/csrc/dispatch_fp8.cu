@@ -13,90 +13,111 @@ namespace {
 constexpr int kThreads = 256;  // register kernel
 
 constexpr int kFp8BulkThreads = 256;
-constexpr int kFp8BulkStages = 2;  // input rows in flight per CTA
-// Cast rows whose bulk stores may still be reading them.  Two (the cast of
-// one token overlapping the stores of the previous one) measured slower at
-// the prefill shape (58.5 vs 54 us alone): the extra stage costs a CTA per
-// SM (5 instead of 6), which hurts more than the overlap helps.
-constexpr int kFp8OutStages = 1;
+#ifndef EP_FP8_IN
+#define EP_FP8_IN 2
+#endif
+#ifndef EP_FP8_OUT
+#define EP_FP8_OUT 1
+#endif
+#ifndef EP_FP8_PARTS
+#define EP_FP8_PARTS 1
+#endif
+constexpr int kFp8InStages = EP_FP8_IN;    // bf16 rows in flight per CTA
+constexpr int kFp8OutStages = EP_FP8_OUT;  // cast rows the bulk stores may still read
+constexpr int kFp8Parts = EP_FP8_PARTS;    // items per token row (when H allows)
 
-// FP8 dispatch through shared memory, one whole token row per item (H a
-// multiple of 512, so both the e4m3 row and its H/128 scales are whole
-// 16-byte units): thread 0 bulk-loads the next token's bf16 row while the
-// CTA quantizes the current one into an output stage (half-warp per
-// 128-channel block), then thread 0 bulk-stores that stage to each of the
-// token's k receive rows (payload and scales).  Bulk stores of whole rows
-// write HBM more efficiently than 8-byte stores per lane.
-__global__ void __launch_bounds__(kFp8BulkThreads)
-    dispatch_fp8_bulk_kernel(const uint4 *__restrict__ x, int T, int H, int k,
+// FP8 dispatch through shared memory, one row part per item (whole rows,
+// or halves when kFp8Parts == 2 and H % 1024 == 0, so that both the e4m3
+// part and its scales are whole 16-byte units): thread 0 bulk-loads the
+// items' bf16 parts kFp8InStages ahead, the CTA quantizes the current one
+// into an output stage (half-warp per 128-channel block), and thread 0
+// bulk-stores that stage to each of the token's k receive rows (codes and
+// scales).  Whole-row bulk stores write HBM better than per-lane stores
+// (measured at the prefill shape: 54 us against 57 us for 16-byte stores
+// per lane and 59 us for 512-byte bulk stores per warp).
+#ifndef EP_FP8_MINB
+#define EP_FP8_MINB 6
+#endif
+__global__ void __launch_bounds__(kFp8BulkThreads, EP_FP8_MINB)
+    dispatch_fp8_bulk_kernel(const uint4 *__restrict__ x, int T, int H, int k, int parts,
                              const int32_t *__restrict__ slot_pos, uint8_t *__restrict__ recv_q,
-                             float *__restrict__ recv_scale, long n_rows, int32_t *d_err) {
+                             float *__restrict__ recv_scale, long n_rows, int first_polls,
+                             int32_t *d_err) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const int in_bytes = 2 * H, q_bytes = H, nb = H >> 7, s_bytes = 4 * nb;
+  const int Hp = H / parts;                                          // channels per item
+  const int in_bytes = 2 * Hp, q_bytes = Hp, nb = H >> 7, nbp = Hp >> 7, s_bytes = 4 * nbp;
   const int out_bytes = q_bytes + s_bytes;                           // a multiple of 16
-  unsigned char *in_buf = smem_raw;                                  // [stages][2H]
-  unsigned char *out_buf = smem_raw + kFp8BulkStages * in_bytes;     // [out stages][H + H/32]
-  __shared__ __align__(8) uint64_t full[kFp8BulkStages];
+  unsigned char *in_buf = smem_raw;                                  // [in stages][2 Hp]
+  unsigned char *out_buf = smem_raw + kFp8InStages * in_bytes;       // [out stages][Hp + Hp/32]
+  __shared__ __align__(8) uint64_t full[kFp8InStages];
   __shared__ int rows[2][EP_MAX_K];
-  __shared__ int timed_out;
   const int tid = threadIdx.x;
-  const long per_cta = (static_cast<long>(T) + gridDim.x - 1) / gridDim.x;
-  const long first = min(static_cast<long>(T), static_cast<long>(blockIdx.x) * per_cta);
-  const long n_mine = min(static_cast<long>(T), first + per_cta) - first;
+  const long items = static_cast<long>(T) * parts;
+  // CTA b takes items [b * per, b * per + per): the CTAs that finish early
+  // leave their SM to the rest (an even split to within one item keeps
+  // every SM's CTAs busy for the same 5-token chains and measured 3 %
+  // slower at the prefill shape)
+  const long per = (items + gridDim.x - 1) / gridDim.x;
+  const long first = min(items, static_cast<long>(blockIdx.x) * per);
+  const long n_mine = min(items, first + per) - first;
 
   // the receive rows are written once and read by a later kernel: evict
   // them first (measured: the step 0.3-0.5 % faster, the kernel ~1 %)
   const uint64_t pol = l2_policy_evict_first();
   if (tid == 0) {
-    for (int s = 0; s < kFp8BulkStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < kFp8InStages; ++s) mbar_init(&full[s], 1);
     mbar_init_fence();
-    timed_out = 0;
   }
   __syncthreads();
   pdl_wait();
 
-  auto issue = [&](long i) {  // thread 0: token first + i -> input stage i % stages
-    const int s = static_cast<int>(i % kFp8BulkStages);
+  auto issue = [&](long i) {  // thread 0: item first + i -> input stage i % stages
+    const int s = static_cast<int>(i % kFp8InStages);
+    const long it = first + i;
+    const long t = it / parts;
+    const int part = static_cast<int>(it - t * parts);
     mbar_arrive_expect_tx(&full[s], in_bytes);
-    bulk_load(in_buf + s * in_bytes, x + (first + i) * (H >> 3), in_bytes, &full[s]);
+    bulk_load(in_buf + s * in_bytes, x + t * (H >> 3) + part * (Hp >> 3), in_bytes, &full[s]);
   };
   if (tid == 0)
-    for (long i = 0; i < min(static_cast<long>(kFp8BulkStages - 1), n_mine); ++i) issue(i);
+    for (long i = 0; i < min(static_cast<long>(kFp8InStages), n_mine); ++i) issue(i);
 
   long i = 0;
+  bool timed_out = false;
   for (; i < n_mine; ++i) {
-    const long t = first + i;
-    const int s = static_cast<int>(i % kFp8BulkStages);
+    const long it = first + i;
+    const long t = it / parts;
+    const int part = static_cast<int>(it - t * parts);
+    const int s = static_cast<int>(i % kFp8InStages);
     unsigned char *out_q = out_buf + (i % kFp8OutStages) * out_bytes;
     float *out_s = reinterpret_cast<float *>(out_q + q_bytes);
-    if (tid == 0) {
-      if (i + kFp8BulkStages - 1 < n_mine) issue(i + kFp8BulkStages - 1);
-      // the stores of the token that last used this output stage have
-      // read it
-      bulk_wait_read<kFp8OutStages - 1>();
-    }
+    // the stores of the item that last used this output stage have read it
+    if (tid == 0) bulk_wait_read<kFp8OutStages - 1>();
     if (tid < k) rows[i & 1][tid] = __ldg(slot_pos + t * k + tid);
-    if (!mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kFp8BulkStages) & 1)))
-      timed_out = 1;
-    __syncthreads();
-    if (timed_out) break;
+    const bool ok = mbar_wait_bounded(&full[s], static_cast<unsigned>((i / kFp8InStages) & 1),
+                                      i == 0 ? first_polls : kMaxBarrierPolls);
+    if (__syncthreads_or(!ok)) {
+      timed_out = true;
+      break;
+    }
     const uint4 *xin = reinterpret_cast<const uint4 *>(in_buf + s * in_bytes);
     uint2 *qo = reinterpret_cast<uint2 *>(out_q);
     // 16 consecutive vectors = one block per half-warp; whole warps share
-    // the loop bound because H / 8 is a multiple of 64
-    for (int v = tid; v < (H >> 3); v += kFp8BulkThreads) {
+    // the loop bound because Hp / 8 is a multiple of 64
+    for (int v = tid; v < (Hp >> 3); v += kFp8BulkThreads) {
       float sc;
       qo[v] = quantize_block_lane(xin[v], &sc);
       if ((tid & 15) == 0) out_s[v >> 4] = sc;
     }
     fence_proxy_async_smem();  // the stage's generic writes before the bulk reads
-    __syncthreads();
+    __syncthreads();           // input stage s read, output stage written
     if (tid == 0) {
+      if (i + kFp8InStages < n_mine) issue(i + kFp8InStages);
       for (int j = 0; j < k; ++j) {
         const int row = rows[i & 1][j];
         if (row < 0 || row >= n_rows) continue;
-        bulk_store(recv_q + static_cast<long>(row) * H, out_q, q_bytes, pol);
-        bulk_store(recv_scale + static_cast<long>(row) * nb, out_s, s_bytes, pol);
+        bulk_store(recv_q + static_cast<long>(row) * H + part * Hp, out_q, q_bytes, pol);
+        bulk_store(recv_scale + static_cast<long>(row) * nb + part * nbp, out_s, s_bytes, pol);
       }
       bulk_commit();
     }
@@ -104,9 +125,11 @@ __global__ void __launch_bounds__(kFp8BulkThreads)
   if (tid == 0) {
     if (timed_out) {
       if (d_err != nullptr) atomicExch(reinterpret_cast<int *>(d_err), EP_ERR_TIMEOUT);
-      for (long q = i + 1; q < min(n_mine, i + kFp8BulkStages); ++q)
-        mbar_wait_bounded(&full[q % kFp8BulkStages],
-                          static_cast<unsigned>((q / kFp8BulkStages) & 1));
+      // the loads still in flight (items i .. i + stages - 1, the one the
+      // wait gave up on included) land before the CTA's memory goes away
+      for (long q = i; q < min(n_mine, i + kFp8InStages); ++q)
+        mbar_wait_bounded(&full[q % kFp8InStages],
+                          static_cast<unsigned>((q / kFp8InStages) & 1));
     }
     bulk_wait<0>();
   }
@@ -185,7 +208,7 @@ __global__ void __launch_bounds__(kThreads)
 // Largest hidden size the bulk FP8 kernel stages in shared memory.
 constexpr int kFp8BulkMaxH = 16384;
 
-int fp8_bulk_smem(int H) { return kFp8BulkStages * 2 * H + kFp8OutStages * (H + H / 32); }
+int fp8_bulk_smem(int Hp) { return kFp8InStages * 2 * Hp + kFp8OutStages * (Hp + Hp / 32); }
 
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
@@ -195,19 +218,21 @@ cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
   // aligned recv_scale
   if (H % 512 == 0 && H <= kFp8BulkMaxH && reinterpret_cast<uintptr_t>(recv_scale) % 16 == 0) {
     if (T == 0) return cudaSuccess;
-    const int smem = fp8_bulk_smem(H);
+    const int parts = (kFp8Parts == 2 && H % 1024 == 0) ? 2 : 1;
+    const int smem = fp8_bulk_smem(H / parts);
     const cudaError_t err =
         raise_dynamic_smem(reinterpret_cast<const void *>(dispatch_fp8_bulk_kernel),
                            fp8_bulk_smem(kFp8BulkMaxH));
     if (err != cudaSuccess) return err;
+    const long items = static_cast<long>(T) * parts;
     const long grid =
         persistent_grid(reinterpret_cast<const void *>(dispatch_fp8_bulk_kernel),
-                        kFp8BulkThreads, smem, static_cast<long>(T) * (kFp8BulkThreads / kWarp),
-                        num_sms);
+                        kFp8BulkThreads, smem, items * (kFp8BulkThreads / kWarp), num_sms);
     ++*launches;
     return launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(kFp8BulkThreads), smem, s, 1,
-                      static_cast<const uint4 *>(x), T, H, k, slot_pos,
-                      static_cast<uint8_t *>(recv_q), recv_scale, n_rows, d_err);
+                      static_cast<const uint4 *>(x), T, H, k, parts, slot_pos,
+                      static_cast<uint8_t *>(recv_q), recv_scale, n_rows, first_wait_polls(),
+                      d_err);
   }
   const long nchunks = (H / 128 + 3) / 4;
   const long items = static_cast<long>(T) * nchunks;

@@ -11,6 +11,7 @@
 #include <tuple>
 #include <utility>
 
+#include "bulk.cuh"
 #include "ep_internal.cuh"
 
 namespace {
@@ -113,6 +114,12 @@ long persistent_grid(const void *kernel, int threads, int smem_bytes, long warp_
   return need < cap ? need : cap;
 }
 
+namespace {
+std::atomic<int> g_first_wait_polls{kMaxBarrierPolls};
+}  // namespace
+
+int first_wait_polls() { return g_first_wait_polls.load(std::memory_order_relaxed); }
+
 cudaError_t raise_dynamic_smem(const void *kernel, int bytes) {
   static std::mutex mu;
   static std::map<std::pair<int, const void *>, int> done;
@@ -136,6 +143,10 @@ int ep_abi_version(void) { return 4; }
 const char *ep_last_error_string(void) { return g_err; }
 
 uint64_t ep_kernel_launches(void) { return g_launches.load(); }
+
+void ep_debug_expire_first_wait(int on) {
+  ep::g_first_wait_polls.store(on ? 0 : ep::kMaxBarrierPolls, std::memory_order_relaxed);
+}
 
 static ep_status_t check_layout_sizes(const char *fn, int T, int k, int E, int R) {
   if (T < 0) return fail(EP_ERR_INVALID_ARG, "%s: T=%d < 0", fn, T);

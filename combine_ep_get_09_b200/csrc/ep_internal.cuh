@@ -73,6 +73,11 @@ cudaError_t launch_pad_layout(const int32_t *cnt_e, const int32_t *slot_pos, int
                               int E, int align, int32_t *off_pad, int32_t *slot_pos_pad,
                               int32_t *recv_src_pad, cudaStream_t s, int *launches);
 
+// Poll limit of the first bounded mbarrier wait of each CTA of the
+// bulk-copy kernels: kMaxBarrierPolls, or 0 while the testing switch
+// ep_debug_expire_first_wait is on.
+int first_wait_polls();
+
 // Sets the message ep_last_error_string() returns on this host thread and
 // returns `status` (for entry points defined outside ep_abi.cu).
 ep_status_t record_error(ep_status_t status, const char *fmt, ...);

@@ -92,6 +92,7 @@ struct FusedArgs {
   float *recv_scale;    // [T*k, H / 128] (FP8)
   int32_t *d_err;
   int per_cta;          // tokens per CTA
+  int first_polls;      // poll limit of each CTA's first row wait
 };
 
 __device__ __forceinline__ void layout_sync() {
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(const FusedAr
     }
   } else if (n_mine > 0) {
     // ---- the first row (warps 8..): wait for it, cast it to FP8 ----
-    ok = mbar_wait_bounded(&full[0], 0u);
+    ok = mbar_wait_bounded(&full[0], 0u, a.first_polls);
     if (kFp8 && ok) {
       cast_row(reinterpret_cast<const uint4 *>(in_buf), out_q, out_s, H, tid - kLayoutThreads,
                kCastThreads);
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
   }
   bool ok = true;
   if (!counts_cta) {
-    ok = mbar_wait_bounded(&full, 0u);
+    ok = mbar_wait_bounded(&full, 0u, a.first_polls);
     if (kFp8 && ok) {
       cast_row(reinterpret_cast<const uint4 *>(in_buf), out_q, out_s, H, tid, kTokThreads);
       fence_proxy_async_smem();  // the stage's generic writes before the bulk reads
@@ -686,6 +687,7 @@ cudaError_t launch_layout_dispatch(const LayoutArgs &la, const void *x, int H, b
   a.recv = static_cast<unsigned char *>(recv);
   a.recv_scale = recv_scale;
   a.d_err = la.d_err;
+  a.first_polls = first_wait_polls();
   ++*launches;
   if (la.id_kind == kIdsInt64)
     return fp8 ? launch_fused<long long, true>(a, num_sms, s)

@@ -22,7 +22,10 @@
  *  - Asynchronous: work is enqueued on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream) and the call returns without waiting.
  *  - Stateless: nothing is kept between calls, so calls on different
- *    streams with different buffers may run concurrently.
+ *    streams with different buffers may run concurrently.  (Two
+ *    exceptions, both described below: ep_get_layout_noalloc shares one
+ *    scratch array per device between its calls, and the testing switch
+ *    ep_debug_expire_first_wait is process-wide.)
  *  - The caller allocates and owns every buffer; the library allocates no
  *    device memory.
  *  - Argument errors are returned before anything is enqueued; nothing is
@@ -349,16 +352,26 @@ ep_status_t ep_map_replicas(const void *idx, int idx_is_int64, int T, int k,
  * example 70000 tokens, top-8 over 128 experts in 16 ranks needs 170 KB
  * and fits.
  *
- * Set-up: the first call on each device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture begins.
+ * Device: the array used is the current device's.  A call that uses it
+ * (the tiled sizes) checks that `stream` belongs to the current device
+ * and that idx is memory the current device can read, and returns
+ * EP_ERR_INVALID_ARG otherwise, before anything is enqueued.
+ *
+ * Set-up: each call that uses the array looks up its device address
+ * (cudaGetSymbolAddress) in the current context -- never a stale one,
+ * whichever context is current.  The first lookup on a device loads the
+ * library's module there; make that first call before any stream capture
+ * begins.
  *
  * Sharing: every call on a device uses the same array, which keeps the
- * last call's contents; each call clears the part that must start at
- * zero (the 16-byte ticket) on `stream` before its kernels run.  Calls
- * whose work overlaps on the GPU (different streams, no ordering between
- * them) race on the array and give wrong layouts: order them on one
- * stream, or use ep_get_layout with one workspace per stream.
+ * last call's contents (it is zero-filled when the module loads).  Each
+ * call clears the part that must start at zero (the 16-byte ticket) with
+ * a 16-byte cudaMemsetAsync on `stream` before its kernels run: a call
+ * that completes leaves the ticket at zero anyway, but one that raced
+ * with another might not, and the clear keeps that from spoiling later
+ * calls.  Calls whose work overlaps on the GPU (different streams, no
+ * ordering between them) race on the array and give wrong layouts: order
+ * them on one stream, or use ep_get_layout with one workspace per stream.
  */
 ep_status_t ep_get_layout_noalloc(const void *idx, int idx_is_int64, int T,
                                   int k, int E, int R, int32_t *cnt_e,
@@ -366,6 +379,23 @@ ep_status_t ep_get_layout_noalloc(const void *idx, int idx_is_int64, int T,
                                   int32_t *off_e, int32_t *off_r,
                                   int32_t *slot_pos, int32_t *recv_src,
                                   int32_t *d_err, void *stream);
+
+/*
+ * ep_debug_expire_first_wait -- testing switch for the bounded waits.
+ *
+ * The bulk-copy kernels (ep_combine and ep_combine_fp8 with k <= 8, the
+ * FP8 ep_dispatch for H % 512 == 0, and both kernels of
+ * ep_layout_dispatch) wait for their own asynchronous copies on shared-
+ * memory barriers, each wait bounded by an iteration limit; when a limit
+ * runs out the kernel records EP_ERR_TIMEOUT in d_err, waits (bounded) for
+ * the copies it still has in flight and returns, leaving its output
+ * incomplete.  With on != 0, the first such wait of every CTA of kernels
+ * launched afterwards gives up at once, without polling, while its copy
+ * still lands normally -- so that path can be run and checked without
+ * making any copy fail.  on == 0 (the default) restores the normal limit.
+ * Process-wide; for tests only (the pages have no counterpart).
+ */
+void ep_debug_expire_first_wait(int on);
 
 /*
  * Waits for `stream` and returns the device error word *d_err (EP_OK when

@@ -5,6 +5,7 @@ import torch
 
 import combine_ep_get_09_b200 as ep
 import oracle
+import workloads
 
 LAYOUT_KEYS = ("cnt_e", "cnt_r", "in_rank", "off_e", "off_r", "slot_pos", "recv_src")
 
@@ -43,3 +44,33 @@ def tensor_bits16(t: torch.Tensor) -> np.ndarray:
 
 def tensor_bytes(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.uint8).cpu().numpy()
+
+
+def assert_scales_equal(got: np.ndarray, want: np.ndarray):
+    """Scale bits equal, except that a NaN scale only has to be a NaN: the
+    reading makes a block with a NaN get a NaN scale, and its payload bits
+    are not part of it (C division keeps the operand's payload, the GPU
+    returns its canonical NaN)."""
+    nan = np.isnan(want)
+    np.testing.assert_array_equal(np.isnan(got), nan)
+    np.testing.assert_array_equal(got.view(np.uint32)[~nan], want.view(np.uint32)[~nan])
+
+
+def nan_inf_batch(cfg, seed, T, H):
+    """A batch whose blocks hold NaNs and infinities (reading c7): a NaN
+    makes its block's amax NaN (it sorts above inf), hence a NaN scale and
+    all codes 0x7f; an infinite amax gives an infinite scale, under which
+    finite values become signed zeros and the infinities NaN (inf / inf)."""
+    b = workloads.make_batch(cfg, seed, T=T, H=H)
+    x = b.x.float()
+    nan, inf = float("nan"), float("inf")
+    x[0, 5] = nan                     # one NaN in block 0
+    x[1, 130] = inf                   # +inf in block 1
+    x[2, 300] = -inf                  # -inf in block 2
+    x[3] = nan                        # a whole row of NaN
+    x[4, 10], x[4, 20] = inf, nan     # both in one block
+    x[6, :128] = inf                  # a block of +inf, then one of -inf
+    x[6, 128:256] = -inf
+    b.x = x.to(torch.bfloat16)
+    b.x.view(torch.int16)[5, H - 7] = -64   # 0xffc0: a NaN with its sign bit set
+    return b

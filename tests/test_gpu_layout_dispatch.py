@@ -12,7 +12,8 @@ import torch
 import combine_ep_get_09_b200 as ep
 import oracle
 import workloads
-from _parity import LAYOUT_KEYS, assert_layout_equal, tensor_bits16, tensor_bytes
+from _parity import (LAYOUT_KEYS, assert_layout_equal, assert_scales_equal,
+                     nan_inf_batch, tensor_bits16, tensor_bytes)
 
 pytestmark = pytest.mark.gpu
 
@@ -78,7 +79,7 @@ def _check(idx, x, E, R, fp8, **kw):
                                       np.full((T * k, H), CANARY8, np.uint8),
                                       np.full((T * k, H // 128), -1.0, np.float32))
         np.testing.assert_array_equal(got["recv"], wq)
-        np.testing.assert_array_equal(got["scale"], ws_.view(np.uint32))
+        assert_scales_equal(got["scale"].view(np.float32), ws_)
     else:
         want = oracle.dispatch_bf16(x, ref["slot_pos"], T * k,
                                     np.full((T * k, H), 0xA5A5, np.uint16))
@@ -187,6 +188,14 @@ def test_fp8_hidden_sizes(H, fused):
 def test_misaligned_scales_take_two_kernels():
     cfg, b = _batch("decode", 18, T=50, H=1024)
     assert _check(b.idx, b.x, cfg.E, cfg.R, True, scale_offset=1) == 2
+
+
+@pytest.mark.parametrize("num_sms", [0, 1])
+def test_fp8_nan_and_inf(num_sms):
+    # all SMs: the one-token-per-CTA kernel; one SM: the token-range kernel
+    cfg = workloads.CONFIGS["decode"]
+    b = nan_inf_batch(cfg, 23, 40, 1024)
+    assert _check(b.idx, b.x, cfg.E, cfg.R, True, num_sms=num_sms) == 1
 
 
 @pytest.mark.parametrize("num_sms", [1, 7, 148])

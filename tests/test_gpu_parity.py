@@ -15,8 +15,8 @@ import torch
 import combine_ep_get_09_b200 as ep
 import oracle
 import workloads
-from _parity import (assert_layout_equal, bf16_ulp_dist, gpu_layout,
-                     tensor_bits16, tensor_bytes)
+from _parity import (assert_layout_equal, assert_scales_equal, bf16_ulp_dist, gpu_layout,
+                     nan_inf_batch, tensor_bits16, tensor_bytes)
 
 pytestmark = pytest.mark.gpu
 
@@ -183,7 +183,7 @@ def _dispatch_fp8_check(cfg, b, num_sms=0):
                                   np.full((T * k, H), CANARY8, np.uint8),
                                   np.full((T * k, H // 128), -1.0, np.float32))
     np.testing.assert_array_equal(tensor_bytes(q), wq)
-    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), ws_.view(np.uint32))
+    assert_scales_equal(s.cpu().numpy(), ws_)
 
 
 @pytest.mark.parametrize("name", ["decode", "prefill", "skewed"])
@@ -212,7 +212,7 @@ def test_dispatch_fp8_misaligned_scales_use_register_path():
     ep.ep_dispatch(b.x.cuda(), L.slot_pos, fp8=True, recv=q, recv_scale=s)
     wq, ws_ = oracle.dispatch_fp8(b.x, ref["slot_pos"], T * k)
     np.testing.assert_array_equal(tensor_bytes(q), wq)
-    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), ws_.view(np.uint32))
+    assert_scales_equal(s.cpu().numpy(), ws_)
 
 
 def test_dispatch_fp8_special_values():
@@ -228,6 +228,15 @@ def test_dispatch_fp8_special_values():
     x[4, :128] = torch.arange(128) * (3.5 / 127)
     x[5, 256:384] = torch.tensor([17.0, 19.0, 9.5, -448.0] * 32) / 128.0
     b.x = x.to(torch.bfloat16)
+    _dispatch_fp8_check(cfg, b)
+
+
+@pytest.mark.parametrize("H", [1024, 896, 7168])
+def test_dispatch_fp8_nan_and_inf(H):
+    # H = 1024 and 7168 fill whole 512-channel groups (one 16-byte scale
+    # store per group and row); H = 896 ends in a partial group
+    cfg = workloads.CONFIGS["decode"]
+    b = nan_inf_batch(cfg, 21, 16, H)
     _dispatch_fp8_check(cfg, b)
 
 

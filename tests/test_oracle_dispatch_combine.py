@@ -116,6 +116,24 @@ def test_dispatch_fp8_nan_propagates():
     assert np.isfinite(s[0, 1]) and not np.any(q[0, 128:] == 0x7F)
 
 
+def test_dispatch_fp8_infinite_amax():
+    # IEEE arithmetic of the stated steps: amax = inf gives s = inf / 448 =
+    # inf; a finite value over inf is a zero of its own sign (e4m3 0x00 /
+    # 0x80) and inf / inf is NaN (0x7f); the next block is untouched
+    x = torch.randn(1, 256).to(torch.bfloat16)
+    x[0, 0] = 2.5
+    x[0, 1] = -3.0
+    x[0, 7] = float("inf")
+    x[0, 9] = float("-inf")
+    q, s = oracle.dispatch_fp8(x, np.array([[0]], np.int32), 1)
+    assert np.isposinf(s[0, 0]) and np.isfinite(s[0, 1])
+    assert q[0, 0] == 0x00 and q[0, 1] == 0x80
+    assert q[0, 7] == 0x7F and q[0, 9] == 0x7F
+    signs = (x[0, :128].float().numpy() < 0)
+    finite = np.isfinite(x[0, :128].float().numpy())
+    assert np.all(q[0, :128][finite] == np.where(signs[finite], 0x80, 0x00))
+
+
 # ------------------------------------------------------------------ combine
 
 def test_combine_hand_worked():
