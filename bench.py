@@ -263,6 +263,19 @@ class Step:
 KERNELS = ("layout", "dispatch_bf16", "dispatch_fp8", "combine")
 
 
+def workload_config(cfg, world: int) -> dict:
+    """The `config` object of both arms: the prefill workload and the step."""
+    return {
+        "workload": ("prefill: T=4096 tokens, H=7168, E=256 experts in R=8 logical ranks, "
+                     "top-8 group-limited routing; step = layout + bf16 dispatch + FP8 "
+                     "dispatch + combine"),
+        "T": cfg.T, "H": cfg.H, "E": cfg.E, "R": cfg.R, "k": cfg.k,
+        "bytes_per_step": sum(step_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R).values()),
+        "l2": "flushed between steps outside the step events: 256 MiB write, then 256 MiB read",
+        "parallelism": f"{world} independent batch(es), one per GPU",
+    }
+
+
 def bench_ours(args, world, rank, device):
     import combine_ep_get_09_b200 as ep
     ep.lib()
@@ -333,16 +346,7 @@ def bench_ours(args, world, rank, device):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": ("prefill: T=4096 tokens, H=7168, E=256 experts in R=8 "
-                         "logical ranks, top-8 group-limited routing; step = "
-                         "layout + bf16 dispatch + FP8 dispatch + combine"),
-            "T": cfg.T, "H": cfg.H, "E": cfg.E, "R": cfg.R, "k": cfg.k,
-            "bytes_per_step": total_bytes,
-            "l2": ("flushed between steps outside the step events: 256 MiB write, "
-                   "then 256 MiB read"),
-            "parallelism": f"{world} independent batch(es), one per GPU",
-        },
+        "config": workload_config(cfg, world),
         "frac_of_8TBs": round(value / world / SPEC_HBM_GBS, 4),
         "kernels": kernels,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
@@ -369,6 +373,19 @@ def bench_ours(args, world, rank, device):
         result["e2e"] = bench_e2e(ep, cfg, batch, device, args, world, total_bytes)
     if world == 1 and rank == 0 and not args.skip_cpu:
         result["cpu_baseline"] = cpu_baseline(cfg, batch, args.cpu_seconds)
+    # the headline figures once more, compactly, at the end of the line
+    summary = {"step_GB/s": result["value"], "step_frac_of_8TBs": result["frac_of_8TBs"],
+               "back_to_back_GB/s": back_to_back["value"],
+               "kernel_us": {n: kernels[n]["us"] for n in KERNELS},
+               "kernel_frac_of_8TBs": {n: kernels[n]["frac_of_8TBs"] for n in KERNELS[1:]}}
+    if "decode" in result:
+        d = result["decode"]
+        warm = next(v for k_, v in d.items() if k_.startswith("us_warm"))
+        summary["decode_us_per_call"] = {
+            "fused_warm_graph": warm["fused_call"], "unfused_warm_graph": warm["unfused_call"],
+            "fused_cold_l2": d["us_cold_l2"]["fused_call"],
+            "unfused_cold_l2": d["us_cold_l2"]["unfused_call"]}
+    result["summary"] = summary
     return result
 
 
@@ -407,21 +424,22 @@ def kernel_source_digest(kernel: str) -> str:
     return h.hexdigest()
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
 def profiled_traffic(kernel: str):
-    """DRAM bytes per launch (read + write) from the committed Nsight Compute
-    summary profiles/<kernel>_prefill.md, or None when there is none or the
-    kernel's sources changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_prefill.md")
+    """DRAM bytes per launch (read + write, one Nsight Compute capture of the
+    prefill workload) recorded for `kernel` in profiles/traffic.json, or
+    None when there is none or the kernel's sources changed since the
+    capture (its recorded source_sha256 differs from the current one)."""
     try:
-        with open(path) as f:
-            text = f.read()
-    except OSError:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
         return None
-    m = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
-    t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m or not t or m.group(1) != kernel_source_digest(kernel):
+    if not rec or rec.get("source_sha256") != kernel_source_digest(kernel):
         return None
-    return float(t.group(1))
+    return float(rec["traffic_bytes_per_launch"])
 
 
 def bench_rank_dedup(ep, st, cfg, device, world, iters=20):
@@ -864,32 +882,61 @@ def bench_overlap(ep, st, cfg, device, world, reps=10):
     return res
 
 
-def bench_decode(ep, device, world, iters=200):
+def bench_decode(ep, device, world, calls=20, reps=10, cold_reps=50):
+    """The 128-token decode workload: µs per call of layout + FP8 dispatch +
+    combine, fused (ep_layout_dispatch + combine, two kernels) and unfused
+    (three kernels), and of each kernel alone.
+
+    warm: `calls` back-to-back calls captured in one CUDA graph and the
+    graph replayed `reps` times (the form a decode step's graph has: the
+    calls overlap their launch latency through programmatic dependent
+    launch, and the graph's own launch is paid once per `calls` calls); the
+    working set stays in L2.  cold: each call alone after the L2 flush,
+    CUDA events right around it on the stream (no graph)."""
     cfg = workloads.CONFIGS["decode"]
     batch = workloads.make_batch(cfg, seed=100)
     st = Step(ep, cfg, batch, device)
     stream = torch.cuda.Stream(device)
+    flush = L2Flush(device)
+    c = cfg
+
+    def layout():
+        ep.ep_get_layout(st.idx, c.E, c.R, out=st.layout, ws=st.ws, d_err=st.d_err,
+                         stream=stream)
+
+    def dispatch_fp8():
+        ep.ep_dispatch(st.x, st.layout.slot_pos, fp8=True, recv=st.recv_q,
+                       recv_scale=st.recv_s, d_err=st.d_err, stream=stream)
+
+    def layout_dispatch():
+        ep.ep_layout_dispatch(st.idx, c.E, c.R, st.x, True, out=st.layout, recv=st.recv_q,
+                              recv_scale=st.recv_s, ws=st.ws, d_err=st.d_err, stream=stream)
+
+    def combine():
+        ep.ep_combine(st.recv, st.layout.slot_pos, st.w, out=st.out, d_err=st.d_err,
+                      stream=stream)
+
+    def unfused():
+        layout()
+        dispatch_fp8()
+        combine()
+
+    def fused():
+        layout_dispatch()
+        combine()
+
     with torch.cuda.stream(stream):
         for _ in range(20):
             st.run(stream, fp8_only=True)
+            fused()
     stream.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        a.record(stream)
-        for _ in range(iters):
-            st.run(stream, fp8_only=True)
-        b.record(stream)
-    stream.synchronize()
-    us_stream = a.elapsed_time(b) * 1e3 / iters
 
-    def graph_us(fn, calls=1):
-        """Device time per call of fn, with `calls` back-to-back calls
-        captured in one CUDA graph and the graph replayed."""
+    def warm_us(fn):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for _ in range(calls):
                 fn()
-        reps = max(1, iters // calls)
         with torch.cuda.stream(stream):
             for _ in range(3):
                 g.replay()
@@ -901,58 +948,38 @@ def bench_decode(ep, device, world, iters=200):
         del g
         return a.elapsed_time(b) * 1e3 / (reps * calls)
 
-    c = cfg
+    def cold_us(fn):
+        evs = []
+        with torch.cuda.stream(stream):
+            for _ in range(cold_reps + 3):
+                flush()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                evs.append((e0, e1))
+        stream.synchronize()
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs[3:]) * 1e3
 
-    def layout_dispatch():
-        ep.ep_layout_dispatch(st.idx, c.E, c.R, st.x, True, out=st.layout, recv=st.recv_q,
-                              recv_scale=st.recv_s, ws=st.ws, d_err=st.d_err, stream=stream)
-
-    def combine():
-        ep.ep_combine(st.recv, st.layout.slot_pos, st.w, out=st.out, d_err=st.d_err,
-                      stream=stream)
-
-    def fused_call():
-        layout_dispatch()
-        combine()
-
-    us_graph = graph_us(lambda: st.run(stream, fp8_only=True))
-    us_fused = graph_us(fused_call)
-    # a decode step's graph holds more than one call: calls in sequence
-    # inside one graph overlap launch latency through programmatic
-    # dependent launch, and the graph's own launch is paid once
-    in_graph = {"unfused": graph_us(lambda: st.run(stream, fp8_only=True), calls=20),
-                "fused": graph_us(fused_call, calls=20)}
-    # each kernel of the call alone, replayed from its own graph
-    parts = {
-        "layout": lambda: ep.ep_get_layout(st.idx, c.E, c.R, out=st.layout, ws=st.ws,
-                                           d_err=st.d_err, stream=stream),
-        "dispatch_fp8": lambda: ep.ep_dispatch(st.x, st.layout.slot_pos, fp8=True,
-                                               recv=st.recv_q, recv_scale=st.recv_s,
-                                               d_err=st.d_err, stream=stream),
-        "layout_dispatch_fp8": layout_dispatch,
-        "combine": combine,
-    }
-    part_us = {name: round(max_over_ranks(graph_us(fn), world, device), 2)
-               for name, fn in parts.items()}
+    fns = {"fused_call": fused, "unfused_call": unfused, "layout": layout,
+           "dispatch_fp8": dispatch_fp8, "layout_dispatch_fp8": layout_dispatch,
+           "combine": combine}
+    warm = {n: round(max_over_ranks(warm_us(f), world, device), 2) for n, f in fns.items()}
+    cold = {n: round(max_over_ranks(cold_us(f), world, device), 2) for n, f in fns.items()}
     if ep.ep_read_error(st.d_err, stream) != 0:
         raise RuntimeError("the device reported an error in the decode calls")
-    us_stream = max_over_ranks(us_stream, world, device)
-    us_graph = max_over_ranks(us_graph, world, device)
-    us_fused = max_over_ranks(us_fused, world, device)
-    in_graph = {name: round(max_over_ranks(v, world, device), 2) for name, v in in_graph.items()}
     nb = decode_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R)
     return {"workload": "decode: T=128, H=7168, E=256/R=8, top-8, FP8 dispatch; "
                         "call = layout + FP8 dispatch + combine",
-            "us_per_call_graph": round(us_graph, 2),
-            "us_per_call_graph_fused": round(us_fused, 2),
-            "fused": "ep_layout_dispatch (layout + FP8 dispatch, one kernel) + combine",
-            "us_per_kernel_graph": part_us,
-            "us_per_call_in_graph_of_20": in_graph,
-            "us_per_call_stream": round(us_stream, 2),
+            "fused": "ep_layout_dispatch (layout + FP8 dispatch, one kernel) + ep_combine",
+            "unfused": "ep_get_layout + ep_dispatch(fp8) + ep_combine",
+            "us_warm_graph_of_%d" % calls: warm,
+            "us_cold_l2": cold,
             "bytes_per_call": nb,
-            "GB/s_graph": round(nb / (us_graph * 1e-6) / 1e9, 1),
-            "GB/s_graph_fused": round(nb / (us_fused * 1e-6) / 1e9, 1),
-            "l2": "warm (back-to-back calls; the working set fits in L2)",
+            "GB/s_warm_fused": round(nb / (warm["fused_call"] * 1e-6) / 1e9, 1),
+            "how": (f"warm: {calls} back-to-back calls (or kernel launches) in one CUDA graph, "
+                    f"replayed {reps} times; cold: median of {cold_reps} single calls, each "
+                    "after the L2 flush, events around the call on its stream"),
             "pages_context_us": 163.0}
 
 
@@ -1032,13 +1059,13 @@ def oracle_sample_step(oracle, cfg, x, idx, w):
     oracle.combine(recv, L["slot_pos"], w)
 
 
-def cpu_baseline(cfg, batch, seconds: float, sample_tokens: int = 512):
+def cpu_baseline(cfg, batch, seconds: float):
+    """The oracle as it stands, single-threaded, on whole steps of the same
+    prefill batch the GPU times (all T tokens), repeated for about
+    `seconds`; then every host core at once (cpu_baseline_threads)."""
     import oracle
-    x = batch.x[:sample_tokens].contiguous()
-    idx = batch.idx[:sample_tokens].contiguous()
-    w = batch.w[:sample_tokens].contiguous()
-    nb = sum(step_bytes(sample_tokens, cfg.H, cfg.k, cfg.E, cfg.R).values())
-    oracle_sample_step(oracle, cfg, x, idx, w)        # warm
+    x, idx, w = batch.x, batch.idx, batch.w
+    nb = sum(step_bytes(batch.T, cfg.H, cfg.k, cfg.E, cfg.R).values())
     reps, t0 = 0, time.perf_counter()
     while True:
         oracle_sample_step(oracle, cfg, x, idx, w)
@@ -1048,33 +1075,31 @@ def cpu_baseline(cfg, batch, seconds: float, sample_tokens: int = 512):
             break
     res = {"value": round(nb * reps / el / 1e9, 3), "unit": "GB/s", "cores": 1,
            "kind": "oracle",
-           "sample": (f"first {sample_tokens} tokens of the prefill batch, whole step "
-                      f"(layout + bf16 dispatch + FP8 dispatch + combine), "
-                      f"{reps} reps in {el:.1f} s, single-threaded C oracle")}
-    res["all_cores"] = cpu_baseline_threads(cfg, batch, seconds, sample_tokens, nb)
+           "sample": (f"the whole {batch.T}-token prefill batch per step (layout + bf16 "
+                      f"dispatch + FP8 dispatch + combine), {reps} steps in {el:.1f} s, "
+                      "single-threaded C oracle")}
+    res["all_cores"] = cpu_baseline_threads(cfg, batch, seconds, nb)
     return res
 
 
-def cpu_baseline_threads(cfg, batch, seconds: float, sample_tokens: int, nb: int,
-                         max_threads: int = 64):
-    """The same oracle step on every host core at once: one Python thread per
-    core (the C oracle runs without the interpreter lock), each on its own
-    `sample_tokens`-token slice of the batch, for about `seconds`."""
+def cpu_baseline_threads(cfg, batch, seconds: float, nb: int, max_threads: int = 64):
+    """The same oracle step on every host core at once: the batch's tokens
+    split into one contiguous slice per core (one Python thread each; the C
+    oracle runs without the interpreter lock), every thread repeating the
+    step on its slice for about `seconds`.  The slices together are the
+    whole batch, so the bytes of one pass over all of them equal one step's."""
     import threading
     import oracle
-    n = max(1, min(len(os.sched_getaffinity(0)), max_threads))
-    n_slices = max(1, batch.x.shape[0] // sample_tokens)
-    slices = []
-    for i in range(min(n, n_slices)):
-        a = i * sample_tokens
-        slices.append(tuple(t[a:a + sample_tokens].contiguous()
-                            for t in (batch.x, batch.idx, batch.w)))
+    n = max(1, min(len(os.sched_getaffinity(0)), max_threads, batch.T))
+    bounds = [batch.T * i // n for i in range(n + 1)]
+    slices = [tuple(t[bounds[i]:bounds[i + 1]].contiguous() for t in (batch.x, batch.idx, batch.w))
+              for i in range(n)]
     reps = [0] * n
     start = threading.Barrier(n + 1)
     stop = time.perf_counter() + 1e9
 
     def work(i):
-        x, idx, w = slices[i % len(slices)]
+        x, idx, w = slices[i]
         start.wait()
         while time.perf_counter() < stop:
             oracle_sample_step(oracle, cfg, x, idx, w)
@@ -1089,27 +1114,25 @@ def cpu_baseline_threads(cfg, batch, seconds: float, sample_tokens: int, nb: int
     for t in threads:
         t.join()
     el = time.perf_counter() - t0
-    total = sum(reps)
-    return {"value": round(nb * total / el / 1e9, 3), "unit": "GB/s", "cores": n,
+    done = sum(reps[i] * (bounds[i + 1] - bounds[i]) for i in range(n)) / batch.T
+    return {"value": round(nb * done / el / 1e9, 3), "unit": "GB/s", "cores": n,
             "kind": "oracle",
-            "sample": (f"{n} threads, each repeating the step on one of {len(slices)} "
-                       f"{sample_tokens}-token slices of the prefill batch; "
-                       f"{total} steps in {el:.1f} s")}
+            "sample": (f"{n} threads, each repeating the step on its own 1/{n} of the "
+                       f"{batch.T}-token prefill batch; {done:.1f} batches' worth in {el:.1f} s")}
 
 
 def bench_reference(args, world, rank):
     """The oracle as it stands, timed on the host cores: same metric, unit
-    and workload, each step a bounded token sample of the prefill batch."""
+    and workload as the GPU arm -- every step is the whole 4096-token
+    prefill batch (layout + bf16 dispatch + FP8 dispatch + combine),
+    single-threaded."""
     if rank != 0:
         return None
     import oracle
     cfg = workloads.CONFIGS["prefill"]
     batch = workloads.make_batch(cfg, seed=0)
-    ns = args.reference_tokens
-    x = batch.x[:ns].contiguous()
-    idx = batch.idx[:ns].contiguous()
-    w = batch.w[:ns].contiguous()
-    nb = sum(step_bytes(ns, cfg.H, cfg.k, cfg.E, cfg.R).values())
+    x, idx, w = batch.x, batch.idx, batch.w
+    nb = sum(step_bytes(cfg.T, cfg.H, cfg.k, cfg.E, cfg.R).values())
     for _ in range(args.warmup):
         oracle_sample_step(oracle, cfg, x, idx, w)
     t0 = time.perf_counter()
@@ -1117,16 +1140,13 @@ def bench_reference(args, world, rank):
         oracle_sample_step(oracle, cfg, x, idx, w)
     el = time.perf_counter() - t0
     value = nb * args.steps / el / 1e9
-    sample = (f"first {ns} tokens of the prefill batch per step (of {cfg.T}); "
-              f"single-threaded C oracle")
+    sample = (f"the whole {cfg.T}-token prefill batch per step, {args.steps} steps after "
+              f"{args.warmup} warm-up steps; single-threaded C oracle")
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": ("prefill: T=4096 tokens, H=7168, E=256 experts in R=8 "
-                                    "logical ranks, top-8 group-limited routing; step = "
-                                    "layout + bf16 dispatch + FP8 dispatch + combine"),
-                       "sample_tokens_per_step": ns},
+            "config": workload_config(cfg, world),
             "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -1134,10 +1154,11 @@ def bench_reference(args, world, rank):
 
 
 def profile_kernel(args, device):
-    """Runs one kernel of the path by itself, --steps times after --warmup
-    warm-ups, with the L2 flush before each launch: the small, repeatable
-    command that Nsight Compute captures are taken on.  Prints the mean
-    CUDA-event time of the kernel (not a benchmark line)."""
+    """Runs one kernel of the path by itself (or, with --profile step, the
+    whole step), --steps times after --warmup warm-ups, with the L2 flush
+    before each launch: the small, repeatable command that Nsight Compute
+    captures are taken on.  Prints the mean CUDA-event time of the call (not
+    a benchmark line)."""
     import combine_ep_get_09_b200 as ep
     cfg = workloads.CONFIGS[args.workload]
     st = Step(ep, cfg, workloads.make_batch(cfg, seed=0), device)
@@ -1160,6 +1181,9 @@ def profile_kernel(args, device):
         "combine_fp8": lambda: ep.ep_combine_fp8(st.recv_q, st.recv_s, st.layout.slot_pos, st.w,
                                                  out=st.out, d_err=st.d_err, stream=stream),
     }
+    # the whole step, for captures of a kernel in the state the previous
+    # kernels of the step leave (with ncu --cache-control none)
+    calls["step"] = lambda: st.run(stream)
     call = calls[args.profile]
     with torch.cuda.stream(stream):
         st.run(stream)
@@ -1198,9 +1222,8 @@ def main():
     p.add_argument("--skip-workloads", action="store_true",
                    help="skip the skewed and large shapes")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
-    p.add_argument("--reference-tokens", type=int, default=256)
     p.add_argument("--profile", choices=("layout", "dispatch_bf16", "dispatch_fp8", "combine",
-                                         "layout_dispatch_fp8", "combine_fp8"),
+                                         "layout_dispatch_fp8", "combine_fp8", "step"),
                    help="run only this kernel (for profiler captures)")
     p.add_argument("--workload", choices=tuple(workloads.CONFIGS), default="prefill",
                    help="workload of --profile")

@@ -28,8 +28,9 @@ def test_source_digest_ignores_comments():
 def test_cpu_baseline_reports_both_legs():
     cfg = workloads.CONFIGS["prefill"]
     batch = workloads.make_batch(cfg, seed=0, T=64, H=256)
-    res = bench.cpu_baseline(cfg, batch, seconds=0.2, sample_tokens=16)
+    res = bench.cpu_baseline(cfg, batch, seconds=0.2)
     assert res["kind"] == "oracle" and res["cores"] == 1 and res["value"] > 0
+    assert "whole 64-token" in res["sample"]
     allc = res["all_cores"]
     assert allc["kind"] == "oracle" and allc["cores"] >= 1 and allc["value"] > 0
     assert "threads" in allc["sample"]

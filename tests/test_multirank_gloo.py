@@ -65,8 +65,7 @@ def test_reference_arm_under_torchrun_prints_once():
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py",
-           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
-           "--reference-tokens", "4"]
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"]
     r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
@@ -75,3 +74,5 @@ def test_reference_arm_under_torchrun_prints_once():
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2
     assert rec["unit"] == "GB/s" and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle"
+    # the same workload as the GPU arm: the whole prefill batch per step
+    assert rec["config"]["T"] == 4096 and rec["config"]["bytes_per_step"] > 1e9
