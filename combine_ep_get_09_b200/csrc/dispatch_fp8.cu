@@ -68,6 +68,14 @@ __global__ void __launch_bounds__(kFp8BulkThreads, EP_FP8_MINB)
     for (int s = 0; s < kFp8InStages; ++s) mbar_init(&full[s], 1);
     mbar_init_fence();
   }
+#ifdef EP_FP8_PF
+  // this CTA's rows into L2 before the wait on the previous kernel (a
+  // prefetch only warms L2)
+  for (long i = tid; i < n_mine; i += kFp8BulkThreads) {
+    const long it = first + i, t = it / parts;
+    prefetch_l2(x + t * (H >> 3) + static_cast<int>(it - t * parts) * (Hp >> 3), in_bytes);
+  }
+#endif
   __syncthreads();
   pdl_wait();
 

@@ -86,6 +86,27 @@ int device_sm_count() {
   return n;
 }
 
+int max_dynamic_smem(const void *kernel) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void *>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 48 << 10;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find({dev, kernel});
+  if (it != cache.end()) return it->second;
+  int optin = 48 << 10;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+      cudaSuccess)
+    optin = 48 << 10;
+  cudaFuncAttributes fa = {};
+  const int stat =
+      cudaFuncGetAttributes(&fa, kernel) == cudaSuccess ? static_cast<int>(fa.sharedSizeBytes)
+                                                        : 1024;
+  const int n = optin - stat;
+  cache[{dev, kernel}] = n;
+  return n;
+}
+
 long persistent_grid(const void *kernel, int threads, int smem_bytes, long warp_items,
                      int num_sms) {
   static std::mutex mu;

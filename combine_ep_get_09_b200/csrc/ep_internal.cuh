@@ -101,6 +101,11 @@ int device_sm_count();
 long persistent_grid(const void *kernel, int threads, int smem_bytes, long warp_items,
                      int num_sms);
 
+// Largest dynamic shared memory a CTA of `kernel` may opt in to on the
+// current device: the device's opt-in limit less the kernel's static shared
+// memory (cached per device and kernel).
+int max_dynamic_smem(const void *kernel);
+
 // Raises a kernel's dynamic shared memory limit to `bytes` (once per
 // device and kernel).
 cudaError_t raise_dynamic_smem(const void *kernel, int bytes);

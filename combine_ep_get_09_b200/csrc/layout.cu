@@ -35,8 +35,14 @@ namespace {
 
 namespace cg = cooperative_groups;
 
+// CTA sizes of the cluster kernel: 512 threads while a CTA's slots fit the
+// warps' registers (at most 4096 slots: 8 chunks of 32 per warp), which
+// leaves room for 128 registers a thread; 1024 above that (64 registers).
+// Measured at the prefill shape (2048 slots a CTA): 512 threads 13.3-13.8
+// us per launch after an L2 flush, 1024 threads 15.0 us.
 constexpr int kClusterThreads = 1024;
-constexpr int kClusterWarps = kClusterThreads / kWarp;
+constexpr int kClusterThreadsSmall = 512;
+constexpr long kClusterSmallCtaSlots = 4096;
 constexpr int kMaxClusterCtas = 16;
 constexpr long kClusterMaxSlots = 1L << 19;
 constexpr long kSlotsPerClusterCta = 2048;  // below this, fewer CTAs
@@ -60,6 +66,7 @@ struct Params {
   unsigned *ticket;  // tiled path
   int32_t *cols;     // tiled path: [ntiles][E + R]
   int tile_T, ntiles;
+  int stage;         // cluster path: the CTA's checked ids live in shared memory
 };
 
 // Expert id from a raw id value: -1 for a dropped or bad slot (a bad one
@@ -350,12 +357,15 @@ __device__ __forceinline__ void cluster_wait() {
 }
 
 // Slots per CTA up to which the CTA's checked ids are kept in shared
-// memory (int16) for the token-mask pass.
-constexpr long kStageIdsMax = 4096;
+// memory (int16) for the token-mask pass, when that fits.
+constexpr long kStageIdsMax = 16384;
 
-int cluster_smem_bytes(int E, int R, int warps, int ctas, long staged_ids) {
+// Shared memory of the cluster kernel: per-warp histograms, every CTA's
+// counts, the lower CTAs' counts, the totals, and (staged) the CTA's
+// checked ids (int16).
+int cluster_smem_bytes(int E, int R, int warps, int ctas, long staged) {
   return (warps * (E + R + 1) + (ctas + 2) * (E + R)) * static_cast<int>(sizeof(int)) +
-         static_cast<int>(((staged_ids * 2 + 15) / 16) * 16);
+         static_cast<int>(((staged * 2 + 15) / 16) * 16);
 }
 
 // Warp-wide exclusive scan of a[0..n) in place (32 elements per round) that
@@ -379,8 +389,65 @@ __device__ int scan_counts(int *a, int n, int32_t *cnt, int32_t *off) {
   return carry;
 }
 
-template <typename IdT>
-__global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Params p) {
+// Exclusive scans, in place and by every thread of the CTA, of a[0..n)
+// and (when b is given) b[0..n), n <= 1024: each warp scans 32-entry
+// chunks, then warps 0 and 1 scan the chunk sums (no serial chain through
+// all n entries).  cnt / off, when given, receive a's entries and
+// exclusive offsets (off[n] = the total).  Warp 2 meanwhile scans the nr
+// rank totals r[] (cnt_r / off_r when given).  Returns a's total (and b's
+// in *b_total).  wsum: 66 ints of shared scratch.  Holds three CTA
+// barriers.
+__device__ int block_scan_counts(int *a, int *b, int n, int32_t *cnt, int32_t *off, int *r,
+                                 int nr, int32_t *cnt_r, int32_t *off_r, int *wsum,
+                                 int *b_total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int nch = (n + 31) / 32;
+  for (int c = w; c < nch; c += nw) {
+    const int i = c * 32 + lane;
+    const int x = i < n ? a[i] : 0;
+    const int ix = warp_inclusive_scan(x);
+    if (i < n) {
+      a[i] = ix - x;
+      if (cnt != nullptr) cnt[i] = x;
+    }
+    if (lane == 31) wsum[c] = ix;
+    if (b != nullptr) {
+      const int y = i < n ? b[i] : 0;
+      const int iy = warp_inclusive_scan(y);
+      if (i < n) b[i] = iy - y;
+      if (lane == 31) wsum[32 + c] = iy;
+    }
+  }
+  __syncthreads();
+  if (w == 0 || (w == 1 && b != nullptr)) {
+    int *ws = wsum + 32 * w;
+    const int v = lane < nch ? ws[lane] : 0;
+    const int iv = warp_inclusive_scan(v);
+    if (lane < nch) ws[lane] = iv - v;
+    if (lane == 31) {
+      wsum[64 + w] = iv;
+      if (w == 0 && off != nullptr) off[n] = iv;
+    }
+  } else if (w == 2) {
+    scan_counts(r, nr, cnt_r, off_r);
+  }
+  __syncthreads();
+  for (int c = w; c < nch; c += nw) {
+    const int i = c * 32 + lane;
+    if (i < n) {
+      a[i] += wsum[c];
+      if (off != nullptr) off[i] = a[i];
+      if (b != nullptr) b[i] += wsum[32 + c];
+    }
+  }
+  const int total = wsum[64];
+  if (b_total != nullptr) *b_total = b != nullptr ? wsum[65] : 0;
+  __syncthreads();
+  return total;
+}
+
+template <typename IdT, int kThreads>
+__global__ void __launch_bounds__(kThreads, 1) layout_cluster_kernel(Params p) {
   cg::cluster_group cluster = cg::this_cluster();
   const int n_ctas = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
@@ -392,8 +459,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
   int *all = hist + nw * ld;       // [ctas][C] every CTA's counts, pushed by each CTA
   int *before = all + n_ctas * C;  // [C] counts of the lower-ranked CTAs
   int *tot = before + C;           // [C] totals, then exclusive offsets
-  short *ids_smem = reinterpret_cast<short *>(tot + C);  // staged ids (small CTAs)
-  __shared__ int s_kept;           // rows in use (all CTAs)
+  short *ids_smem = reinterpret_cast<short *>(tot + C);  // staged ids
+  __shared__ int wsum[66];
   const IdT *idx = static_cast<const IdT *>(p.idx);
 
   const int per_cta = (p.T + n_ctas - 1) / n_ctas;
@@ -401,7 +468,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
   const int t_end = min(p.T, t_beg + per_cta);
   const long s_beg = static_cast<long>(t_beg) * p.k;
   const long n = static_cast<long>(t_end - t_beg) * p.k;
-  const bool stage = static_cast<long>(per_cta) * p.k <= kStageIdsMax;
+  const bool stage = p.stage != 0;
 
   for (int i = tid; i < nw * ld; i += nt) smem[i] = 0;
   __syncthreads();
@@ -446,23 +513,18 @@ __global__ void __launch_bounds__(kClusterThreads, 1) layout_cluster_kernel(Para
     }
   }
   __syncthreads();
-  // warp 0 scans the expert totals, warp 1 the rank totals; CTA 0 writes
-  // the counts and offsets as it goes
-  if (w == 0) {
-    const int n_kept =
-        scan_counts(tot, E, rank == 0 ? p.cnt_e : nullptr, rank == 0 ? p.off_e : nullptr);
-    if (tid == 0) s_kept = n_kept;
-  } else if (w == 1) {
-    scan_counts(tot + E, R, rank == 0 ? p.cnt_r : nullptr, rank == 0 ? p.off_r : nullptr);
-  }
-  __syncthreads();
+  // exclusive scans of the expert totals (their offsets; CTA 0 writes
+  // them with the counts) and of the rank totals
+  const int n_kept = block_scan_counts(
+      tot, nullptr, E, rank == 0 ? p.cnt_e : nullptr, rank == 0 ? p.off_e : nullptr, tot + E, R,
+      rank == 0 ? p.cnt_r : nullptr, rank == 0 ? p.off_r : nullptr, wsum, nullptr);
   // row = this warp's count of earlier slots + the CTA's offset in the
   // expert (before) + the expert's offset (tot)
   place_segment(idx, s_beg + seg_beg, s_beg + seg_end, p.k, E, hist + w * ld, sr, p.slot_pos,
                 p.recv_src, before, tot);
   // rows nobody fills (past the kept ones)
   const long N = static_cast<long>(p.T) * p.k;
-  for (long r = s_kept + static_cast<long>(rank) * nt + tid; r < N;
+  for (long r = n_kept + static_cast<long>(rank) * nt + tid; r < N;
        r += static_cast<long>(n_ctas) * nt)
     p.recv_src[r] = -1;
 }
@@ -631,7 +693,9 @@ bool cluster_path(int T, int k) { return static_cast<long>(T) * k <= kClusterMax
 
 // Largest cluster (<= 16 CTAs) the device can schedule for this kernel with
 // `smem` bytes per CTA; cached per (device, id type, smem size).
-template <typename IdT>
+// Largest cluster (16, else the portable 8) the GPU can run with CTAs of
+// kThreads threads and `smem` bytes of dynamic shared memory.
+template <typename IdT, int kThreads>
 int max_cluster_ctas(int smem) {
   static std::mutex mu;
   static std::map<std::pair<int, int>, int> cache;
@@ -640,13 +704,13 @@ int max_cluster_ctas(int smem) {
   std::lock_guard<std::mutex> lock(mu);
   auto it = cache.find({dev, smem});
   if (it != cache.end()) return it->second;
-  auto kern = layout_cluster_kernel<IdT>;
+  auto kern = layout_cluster_kernel<IdT, kThreads>;
   int best = 8;  // portable cluster size
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
       cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kMaxClusterCtas);
-    cfg.blockDim = dim3(kClusterThreads);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
@@ -664,27 +728,45 @@ int max_cluster_ctas(int smem) {
   return best;
 }
 
+// One launch of the cluster kernel with CTAs of kThreads threads: up to 16
+// CTAs of at least kSlotsPerClusterCta slots each (fewer for small
+// batches), the CTA's ids staged in shared memory when they fit.
+template <typename IdT, int kThreads>
+cudaError_t launch_cluster_with(Params p, int n_ctas, cudaStream_t s, int *launches) {
+  auto kern = layout_cluster_kernel<IdT, kThreads>;
+  const int smem_max = max_dynamic_smem(reinterpret_cast<const void *>(kern));
+  const cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern), smem_max);
+  if (err != cudaSuccess) return err;
+  constexpr int warps = kThreads / kWarp;
+  if (n_ctas > 8)
+    n_ctas = min(n_ctas, max_cluster_ctas<IdT, kThreads>(
+                             cluster_smem_bytes(p.E, p.R, warps, kMaxClusterCtas, 0)));
+  const long per_cta_slots = static_cast<long>((p.T + n_ctas - 1) / n_ctas) * p.k;
+  int smem = cluster_smem_bytes(p.E, p.R, warps, n_ctas, 0);
+  p.stage = 0;
+  if (per_cta_slots <= kStageIdsMax) {
+    const int staged = cluster_smem_bytes(p.E, p.R, warps, n_ctas, per_cta_slots);
+    if (staged <= smem_max) {
+      smem = staged;
+      p.stage = 1;
+    }
+  }
+  ++*launches;
+  return launch_pdl(kern, dim3(n_ctas), dim3(kThreads), smem, s, n_ctas, p);
+}
+
 template <typename IdT>
 cudaError_t launch_cluster(Params p, cudaStream_t s, int *launches) {
-  auto kern = layout_cluster_kernel<IdT>;
   const long N = static_cast<long>(p.T) * p.k;
-  const int threads = N <= kSmallSlots ? kSmallThreads : kClusterThreads;
-  cudaError_t err = raise_dynamic_smem(
-      reinterpret_cast<const void *>(kern),
-      cluster_smem_bytes(p.E, p.R, kClusterWarps, kMaxClusterCtas, kStageIdsMax));
-  if (err != cudaSuccess) return err;
+  if (N <= kSmallSlots) return launch_cluster_with<IdT, kSmallThreads>(p, 1, s, launches);
   long want = (N + kSlotsPerClusterCta - 1) / kSlotsPerClusterCta;
-  if (want < 1) want = 1;
-  const int cap = want > 8 ? max_cluster_ctas<IdT>(cluster_smem_bytes(
-                                 p.E, p.R, threads / kWarp, kMaxClusterCtas, kStageIdsMax))
-                           : 8;
-  const int n_ctas = static_cast<int>(want < cap ? want : cap);
-  // slots of the largest CTA: staged in shared memory when small enough
+  const int n_ctas = static_cast<int>(want < kMaxClusterCtas ? want : kMaxClusterCtas);
+  // CTA size from the slots a CTA gets with the full cluster (a smaller
+  // cluster only happens where 16 CTAs cannot run at once)
   const long per_cta_slots = static_cast<long>((p.T + n_ctas - 1) / n_ctas) * p.k;
-  const int smem = cluster_smem_bytes(p.E, p.R, threads / kWarp, n_ctas,
-                                      per_cta_slots <= kStageIdsMax ? per_cta_slots : 0);
-  ++*launches;
-  return launch_pdl(kern, dim3(n_ctas), dim3(threads), smem, s, n_ctas, p);
+  if (per_cta_slots <= kClusterSmallCtaSlots)
+    return launch_cluster_with<IdT, kClusterThreadsSmall>(p, n_ctas, s, launches);
+  return launch_cluster_with<IdT, kClusterThreads>(p, n_ctas, s, launches);
 }
 
 template <typename IdT>
