@@ -894,7 +894,7 @@ def bench_overlap(ep, st, cfg, device, world, reps=10):
     return res
 
 
-def bench_decode(ep, device, world, calls=20, reps=10, cold_reps=50):
+def bench_decode(ep, device, world, calls=20, reps=10, cold_reps=10):
     """The 128-token decode workload: µs per call of layout + FP8 dispatch +
     combine, fused (ep_layout_dispatch + combine, two kernels) and unfused
     (three kernels), and of each kernel alone.
@@ -903,8 +903,10 @@ def bench_decode(ep, device, world, calls=20, reps=10, cold_reps=50):
     graph replayed `reps` times (the form a decode step's graph has: the
     calls overlap their launch latency through programmatic dependent
     launch, and the graph's own launch is paid once per `calls` calls); the
-    working set stays in L2.  cold: each call alone after the L2 flush,
-    CUDA events right around it on the stream (no graph)."""
+    working set stays in L2.  cold: `cold_reps` pairs of (L2 flush, call) in
+    one graph, less the same graph without the calls, per call (single
+    calls timed with their own events read in steps of about 1-2 us on this
+    part)."""
     cfg = workloads.CONFIGS["decode"]
     batch = workloads.make_batch(cfg, seed=100)
     st = Step(ep, cfg, batch, device)
@@ -960,18 +962,32 @@ def bench_decode(ep, device, world, calls=20, reps=10, cold_reps=50):
         del g
         return a.elapsed_time(b) * 1e3 / (reps * calls)
 
-    def cold_us(fn):
-        evs = []
+    def graph_total_us(body):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            body()
         with torch.cuda.stream(stream):
-            for _ in range(cold_reps + 3):
-                flush()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                fn()
-                e1.record(stream)
-                evs.append((e0, e1))
+            g.replay()
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            b.record(stream)
         stream.synchronize()
-        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs[3:]) * 1e3
+        del g
+        return a.elapsed_time(b) * 1e3 / reps
+
+    def flushes():
+        for _ in range(cold_reps):
+            flush()
+
+    flush_us = graph_total_us(flushes)
+
+    def cold_us(fn):
+        def body():
+            for _ in range(cold_reps):
+                flush()
+                fn()
+        return (graph_total_us(body) - flush_us) / cold_reps
 
     fns = {"fused_call": fused, "unfused_call": unfused, "layout": layout,
            "dispatch_fp8": dispatch_fp8, "layout_dispatch_fp8": layout_dispatch,
@@ -990,8 +1006,8 @@ def bench_decode(ep, device, world, calls=20, reps=10, cold_reps=50):
             "bytes_per_call": nb,
             "GB/s_warm_fused": round(nb / (warm["fused_call"] * 1e-6) / 1e9, 1),
             "how": (f"warm: {calls} back-to-back calls (or kernel launches) in one CUDA graph, "
-                    f"replayed {reps} times; cold: median of {cold_reps} single calls, each "
-                    "after the L2 flush, events around the call on its stream"),
+                    f"replayed {reps} times; cold: {cold_reps} (L2 flush, call) pairs in one "
+                    "graph less the flushes alone, per call"),
             "pages_context_us": 163.0}
 
 

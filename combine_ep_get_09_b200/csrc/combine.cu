@@ -34,18 +34,15 @@ namespace {
 constexpr int kRegThreads = 256;
 constexpr int kSlotBatch = 8;    // slot rows loaded together (register path)
 constexpr int kBulkMaxK = 8;     // slot rows one bulk stage holds
-#ifndef EP_COMBINE_STAGES
-#define EP_COMBINE_STAGES 2
-#endif
-#ifndef EP_COMBINE_CHV
-#define EP_COMBINE_CHV 256
-#endif
-constexpr int kStages = EP_COMBINE_STAGES;       // items in flight per CTA
+// Items in flight per CTA.  Deeper rings measured slower at the prefill
+// shape (alone: 77.8 us with 2 stages of 4 KB chunks, 82.0 with 3 stages
+// of 2 KB, 88.1 with 3 of 4 KB, 141 with one CTA per SM and 6 stages).
+constexpr int kStages = 2;
 // 16-byte vectors per row chunk (= threads of the bulk kernel): 256 in
 // general; 64 when every item of the smaller chunks still gets a CTA of its
 // own in one wave (a decode batch), which shortens each CTA's chain.  (128
 // fits one wave only where 64 does too: 6 of its CTAs fit an SM, 13 of 64's.)
-constexpr int kChunkVec = EP_COMBINE_CHV;
+constexpr int kChunkVec = 256;
 constexpr int kSmallChunkVec = 64;
 template <int CHV>
 constexpr int bulk_smem() { return kStages * kBulkMaxK * CHV * 16; }

@@ -13,46 +13,39 @@ namespace {
 constexpr int kThreads = 256;  // register kernel
 
 constexpr int kFp8BulkThreads = 256;
-#ifndef EP_FP8_IN
-#define EP_FP8_IN 2
-#endif
-#ifndef EP_FP8_OUT
-#define EP_FP8_OUT 1
-#endif
-#ifndef EP_FP8_PARTS
-#define EP_FP8_PARTS 1
-#endif
-constexpr int kFp8InStages = EP_FP8_IN;    // bf16 rows in flight per CTA
-constexpr int kFp8OutStages = EP_FP8_OUT;  // cast rows the bulk stores may still read
-constexpr int kFp8Parts = EP_FP8_PARTS;    // items per token row (when H allows)
+constexpr int kFp8InStages = 2;   // bf16 rows in flight per CTA
+// Cast rows whose bulk stores may still be reading them.  Two measured
+// slower at the prefill shape (59.5 vs 57.5 us alone): the extra stage
+// costs a CTA per SM (5 instead of 6), which hurts more than the overlap
+// helps; so did one input stage with two or three output stages (63.5 and
+// 59.4 us).
+constexpr int kFp8OutStages = 1;
 
-// FP8 dispatch through shared memory, one row part per item (whole rows,
-// or halves when kFp8Parts == 2 and H % 1024 == 0, so that both the e4m3
-// part and its scales are whole 16-byte units): thread 0 bulk-loads the
-// items' bf16 parts kFp8InStages ahead, the CTA quantizes the current one
-// into an output stage (half-warp per 128-channel block), and thread 0
-// bulk-stores that stage to each of the token's k receive rows (codes and
-// scales).  Whole-row bulk stores write HBM better than per-lane stores
-// (measured at the prefill shape: 54 us against 57 us for 16-byte stores
-// per lane and 59 us for 512-byte bulk stores per warp).
-#ifndef EP_FP8_MINB
-#define EP_FP8_MINB 6
-#endif
-__global__ void __launch_bounds__(kFp8BulkThreads, EP_FP8_MINB)
-    dispatch_fp8_bulk_kernel(const uint4 *__restrict__ x, int T, int H, int k, int parts,
+// FP8 dispatch through shared memory, one token row per item (H a
+// multiple of 512, so that both the e4m3 row and its H/128 scales are
+// whole 16-byte units): thread 0 bulk-loads the rows kFp8InStages ahead,
+// the CTA quantizes the current one into an output stage (half-warp per
+// 128-channel block), and thread 0 bulk-stores that stage to each of the
+// token's k receive rows (codes and scales).  Whole-row bulk stores write
+// HBM better than per-lane stores (measured at the prefill shape: 55 us
+// against 57 us for 16-byte stores per lane, 59 us for 512-byte bulk
+// stores per warp, and 61 us for half-row items).
+// 6 CTAs of 256 threads fit an SM's shared memory at H = 7168; the bound
+// keeps registers at or below 42 so that they fit too.
+__global__ void __launch_bounds__(kFp8BulkThreads, 6)
+    dispatch_fp8_bulk_kernel(const uint4 *__restrict__ x, int T, int H, int k,
                              const int32_t *__restrict__ slot_pos, uint8_t *__restrict__ recv_q,
                              float *__restrict__ recv_scale, long n_rows, int first_polls,
                              int32_t *d_err) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const int Hp = H / parts;                                          // channels per item
-  const int in_bytes = 2 * Hp, q_bytes = Hp, nb = H >> 7, nbp = Hp >> 7, s_bytes = 4 * nbp;
+  const int in_bytes = 2 * H, q_bytes = H, nb = H >> 7, s_bytes = 4 * nb;
   const int out_bytes = q_bytes + s_bytes;                           // a multiple of 16
-  unsigned char *in_buf = smem_raw;                                  // [in stages][2 Hp]
-  unsigned char *out_buf = smem_raw + kFp8InStages * in_bytes;       // [out stages][Hp + Hp/32]
+  unsigned char *in_buf = smem_raw;                                  // [in stages][2H]
+  unsigned char *out_buf = smem_raw + kFp8InStages * in_bytes;       // [out stages][H + H/32]
   __shared__ __align__(8) uint64_t full[kFp8InStages];
   __shared__ int rows[2][EP_MAX_K];
   const int tid = threadIdx.x;
-  const long items = static_cast<long>(T) * parts;
+  const long items = T;
   // CTA b takes items [b * per, b * per + per): the CTAs that finish early
   // leave their SM to the rest (an even split to within one item keeps
   // every SM's CTAs busy for the same 5-token chains and measured 3 %
@@ -68,24 +61,13 @@ __global__ void __launch_bounds__(kFp8BulkThreads, EP_FP8_MINB)
     for (int s = 0; s < kFp8InStages; ++s) mbar_init(&full[s], 1);
     mbar_init_fence();
   }
-#ifdef EP_FP8_PF
-  // this CTA's rows into L2 before the wait on the previous kernel (a
-  // prefetch only warms L2)
-  for (long i = tid; i < n_mine; i += kFp8BulkThreads) {
-    const long it = first + i, t = it / parts;
-    prefetch_l2(x + t * (H >> 3) + static_cast<int>(it - t * parts) * (Hp >> 3), in_bytes);
-  }
-#endif
   __syncthreads();
   pdl_wait();
 
-  auto issue = [&](long i) {  // thread 0: item first + i -> input stage i % stages
+  auto issue = [&](long i) {  // thread 0: token first + i -> input stage i % stages
     const int s = static_cast<int>(i % kFp8InStages);
-    const long it = first + i;
-    const long t = it / parts;
-    const int part = static_cast<int>(it - t * parts);
     mbar_arrive_expect_tx(&full[s], in_bytes);
-    bulk_load(in_buf + s * in_bytes, x + t * (H >> 3) + part * (Hp >> 3), in_bytes, &full[s]);
+    bulk_load(in_buf + s * in_bytes, x + (first + i) * (H >> 3), in_bytes, &full[s]);
   };
   if (tid == 0)
     for (long i = 0; i < min(static_cast<long>(kFp8InStages), n_mine); ++i) issue(i);
@@ -93,9 +75,7 @@ __global__ void __launch_bounds__(kFp8BulkThreads, EP_FP8_MINB)
   long i = 0;
   bool timed_out = false;
   for (; i < n_mine; ++i) {
-    const long it = first + i;
-    const long t = it / parts;
-    const int part = static_cast<int>(it - t * parts);
+    const long t = first + i;
     const int s = static_cast<int>(i % kFp8InStages);
     unsigned char *out_q = out_buf + (i % kFp8OutStages) * out_bytes;
     float *out_s = reinterpret_cast<float *>(out_q + q_bytes);
@@ -111,8 +91,8 @@ __global__ void __launch_bounds__(kFp8BulkThreads, EP_FP8_MINB)
     const uint4 *xin = reinterpret_cast<const uint4 *>(in_buf + s * in_bytes);
     uint2 *qo = reinterpret_cast<uint2 *>(out_q);
     // 16 consecutive vectors = one block per half-warp; whole warps share
-    // the loop bound because Hp / 8 is a multiple of 64
-    for (int v = tid; v < (Hp >> 3); v += kFp8BulkThreads) {
+    // the loop bound because H / 8 is a multiple of 64
+    for (int v = tid; v < (H >> 3); v += kFp8BulkThreads) {
       float sc;
       qo[v] = quantize_block_lane(xin[v], &sc);
       if ((tid & 15) == 0) out_s[v >> 4] = sc;
@@ -124,8 +104,8 @@ __global__ void __launch_bounds__(kFp8BulkThreads, EP_FP8_MINB)
       for (int j = 0; j < k; ++j) {
         const int row = rows[i & 1][j];
         if (row < 0 || row >= n_rows) continue;
-        bulk_store(recv_q + static_cast<long>(row) * H + part * Hp, out_q, q_bytes, pol);
-        bulk_store(recv_scale + static_cast<long>(row) * nb + part * nbp, out_s, s_bytes, pol);
+        bulk_store(recv_q + static_cast<long>(row) * H, out_q, q_bytes, pol);
+        bulk_store(recv_scale + static_cast<long>(row) * nb, out_s, s_bytes, pol);
       }
       bulk_commit();
     }
@@ -139,7 +119,10 @@ __global__ void __launch_bounds__(kFp8BulkThreads, EP_FP8_MINB)
         mbar_wait_bounded(&full[q % kFp8InStages],
                           static_cast<unsigned>((q / kFp8InStages) & 1));
     }
-    bulk_wait<0>();
+    // the stores must have read the output stage before the CTA's shared
+    // memory goes away; their writes are visible to later kernels once the
+    // grid completes
+    bulk_wait_read<0>();
   }
 }
 
@@ -216,7 +199,7 @@ __global__ void __launch_bounds__(kThreads)
 // Largest hidden size the bulk FP8 kernel stages in shared memory.
 constexpr int kFp8BulkMaxH = 16384;
 
-int fp8_bulk_smem(int Hp) { return kFp8InStages * 2 * Hp + kFp8OutStages * (Hp + Hp / 32); }
+int fp8_bulk_smem(int H) { return kFp8InStages * 2 * H + kFp8OutStages * (H + H / 32); }
 
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
@@ -226,19 +209,18 @@ cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
   // aligned recv_scale
   if (H % 512 == 0 && H <= kFp8BulkMaxH && reinterpret_cast<uintptr_t>(recv_scale) % 16 == 0) {
     if (T == 0) return cudaSuccess;
-    const int parts = (kFp8Parts == 2 && H % 1024 == 0) ? 2 : 1;
-    const int smem = fp8_bulk_smem(H / parts);
+    const int smem = fp8_bulk_smem(H);
     const cudaError_t err =
         raise_dynamic_smem(reinterpret_cast<const void *>(dispatch_fp8_bulk_kernel),
                            fp8_bulk_smem(kFp8BulkMaxH));
     if (err != cudaSuccess) return err;
-    const long items = static_cast<long>(T) * parts;
     const long grid =
         persistent_grid(reinterpret_cast<const void *>(dispatch_fp8_bulk_kernel),
-                        kFp8BulkThreads, smem, items * (kFp8BulkThreads / kWarp), num_sms);
+                        kFp8BulkThreads, smem, static_cast<long>(T) * (kFp8BulkThreads / kWarp),
+                        num_sms);
     ++*launches;
     return launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(kFp8BulkThreads), smem, s, 1,
-                      static_cast<const uint4 *>(x), T, H, k, parts, slot_pos,
+                      static_cast<const uint4 *>(x), T, H, k, slot_pos,
                       static_cast<uint8_t *>(recv_q), recv_scale, n_rows, first_wait_polls(),
                       d_err);
   }

@@ -38,46 +38,6 @@ __device__ __forceinline__ uint2 quantize_bf16x8(uint4 v, float s) {
   return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
 }
 
-// The same codes from r = RN(1 / s) instead of a division per value.
-//
-// p = RN(x * r) is within 3 fp32 steps of q = RN(x / s): with u = 2^-24,
-// r = (1/s)(1 + d1) and p = x r (1 + d2), |d1|, |d2| <= u, while
-// q = (x/s)(1 + d3), |d3| <= u, so |p - q| <= (3u + u^2)|x/s|, and an fp32
-// step near |x/s| is at least u |x/s| (for x/s and r normal; a quotient
-// below the normal range lies far below the smallest e4m3 subnormal, whose
-// codes are zero on both sides).  The e4m3 conversion is monotone in the
-// magnitude, so when the codes of |p| four steps down and four steps up
-// agree, that code is q's; otherwise (about one value in 10^5, and every
-// NaN or infinite product) the value takes the IEEE division.  The sign
-// goes on unchanged: e4m3 is sign-magnitude and round-to-nearest-even is
-// symmetric.
-__device__ __forceinline__ uint32_t e4m3x2_bits(float a, float b) {
-  return static_cast<uint32_t>(
-      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
-}
-
-__device__ __forceinline__ uint2 quantize_bf16x8_rcp(uint4 v, float s, float r) {
-  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-  uint32_t q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float lo = __uint_as_float(in[i] << 16);
-    const float hi = __uint_as_float(in[i] & 0xffff0000u);
-    const uint32_t b0 = __float_as_uint(__fmul_rn(lo, r));
-    const uint32_t b1 = __float_as_uint(__fmul_rn(hi, r));
-    const uint32_t m0 = b0 & 0x7fffffffu, m1 = b1 & 0x7fffffffu;
-    const uint32_t down = e4m3x2_bits(__uint_as_float(max(m0, 4u) - 4u),
-                                      __uint_as_float(max(m1, 4u) - 4u));
-    const uint32_t up = e4m3x2_bits(__uint_as_float(m0 + 4u), __uint_as_float(m1 + 4u));
-    if (down == up) {
-      q[i] = down | ((b0 >> 24) & 0x80u) | ((b1 >> 16) & 0x8000u);
-    } else {
-      q[i] = e4m3x2_bits(__fdiv_rn(lo, s), __fdiv_rn(hi, s));
-    }
-  }
-  return make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
-}
-
 // amax -> scale -> e4m3 for the 8 bf16 values of one lane, the lane being
 // one of the 16 lanes (a half-warp) that hold a 128-channel block.
 __device__ __forceinline__ uint2 quantize_block_lane(uint4 v, float *scale) {
@@ -87,11 +47,7 @@ __device__ __forceinline__ uint2 quantize_block_lane(uint4 v, float *scale) {
   float a = __uint_as_float(m << 16);
   a = a < 1e-4f ? 1e-4f : a;  // keeps NaN
   *scale = __fdiv_rn(a, 448.0f);
-#ifdef EP_FP8_RCP
-  return quantize_bf16x8_rcp(v, *scale, __frcp_rn(*scale));
-#else
   return quantize_bf16x8(v, *scale);
-#endif
 }
 
 }  // namespace ep

@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kThreads) layout_dispatch_kernel(const FusedAr
       if (tid == 0 && i + kStages < n_mine) issue(i + kStages);
     }
   }
-  if (tid < k) bulk_wait<0>();
+  if (tid < k) bulk_wait_read<0>();  // stages read before the CTA exits
   if (tid == 0 && timed_out) {
     if (a.d_err != nullptr) atomicExch(reinterpret_cast<int *>(a.d_err), EP_ERR_TIMEOUT);
     // let the row loads still in flight land before the CTA's memory goes away
@@ -608,7 +608,7 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
         bulk_store(a.recv + static_cast<long>(row) * 2 * H, in_buf, 2 * H);
       }
       bulk_commit();
-      bulk_wait<0>();
+      bulk_wait_read<0>();  // the stage read before the CTA exits
     }
   }
 }
