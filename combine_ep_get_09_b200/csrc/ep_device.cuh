@@ -46,12 +46,15 @@ __device__ __forceinline__ void st_stream_f32(float *p, float v) {
 // while the previous kernel on the stream is still finishing; it must call
 // pdl_wait() before touching memory that kernel writes (griddepcontrol.wait
 // returns once the previous grid has completed and its writes are visible;
-// with no such predecessor it returns at once).  No kernel issues
+// with no such predecessor it returns at once).  Almost no kernel issues
 // griddepcontrol.launch_dependents: a CTA's exit counts as its trigger, so
 // the next kernel is launched as this one's last CTAs leave, which hides
 // its launch latency without parking its CTAs on SMs that are still busy.
 // (Triggering at kernel entry measured slower everywhere: 288 vs 256 us
 // for a back-to-back prefill step, 8.23 vs 8.12 us for a decode call.)
+// The one exception, the one-token-per-CTA fused decode kernel, triggers
+// once only its final stores are left (layout_dispatch.cu).
+//
 // Bulk prefetch of [p, p + bytes) into L2 (p 16-byte aligned, bytes a
 // multiple of 16); a hint with no completion to wait for.
 __device__ __forceinline__ void prefetch_l2(const void *p, int bytes) {

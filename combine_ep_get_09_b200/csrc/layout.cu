@@ -644,6 +644,11 @@ __global__ void __launch_bounds__(kTileThreads) layout_count_kernel(Params p) {
 template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads) layout_place_kernel(Params p) {
   pdl_wait();
+  // every count tile is done with the ticket: leave it at zero for the next
+  // call on this workspace, whatever value it has (a completed count kernel
+  // leaves zero anyway, through the wrap of atomicInc; two calls that
+  // overlapped on one workspace might not)
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.ticket = 0u;
   extern __shared__ int smem[];
   const int E = p.E, C = p.E + p.R, ld = hist_ld(p);
   const int tid = threadIdx.x, w = tid >> 5;

@@ -438,6 +438,14 @@ __device__ void token_cta_exclusive_scan(const int *in, int *out, int n, int *wa
   }
 }
 
+// Lets the next kernel on the stream be scheduled before this CTA exits
+// (programmatic dependent launch).  Used only where a CTA's remaining work
+// is its final stores: triggering earlier parks the next kernel's CTAs on
+// SMs that are still busy.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 template <typename IdT, bool kFp8>
 __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(const FusedArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -593,6 +601,11 @@ __global__ void __launch_bounds__(kTokThreads) layout_dispatch_token_kernel(cons
       a.in_rank[static_cast<long>(t) * R + r] = static_cast<uint8_t>(in);
     }
   }
+  // nothing is left but the stores: the next kernel on the stream may be
+  // scheduled now (it still waits for this grid's completion before it
+  // reads anything), which hides its launch behind this CTA's stores
+  // (decode call 8.22 -> 8.01 us in graphs of 20)
+  pdl_trigger();
   if (warp == 0 && lane < k) {
     int before = 0;
     for (int v = 0; v < kTokWarps; ++v) before += part[v][lane];

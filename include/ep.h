@@ -39,10 +39,13 @@
  *  - Pointers must be 16-byte aligned unless stated otherwise.
  *  - Kernels are launched with programmatic stream serialization: one may
  *    be scheduled as the previous kernel on `stream` finishes, and it waits
- *    for that kernel (griddepcontrol.wait) before reading anything.  None
- *    releases its successor early.  A caller's kernel launched after one of
- *    these with the same attribute must wait the same way before reading
- *    their output; one launched without it sees plain stream order.
+ *    for that kernel (griddepcontrol.wait) before reading anything.  Only
+ *    the one-token-per-CTA kernel of ep_layout_dispatch releases its
+ *    successor early, once its CTAs have only their final stores left; the
+ *    successor must still wait before reading.  A caller's kernel launched
+ *    after one of these with the same attribute must wait the same way
+ *    before reading their output; one launched without it sees plain
+ *    stream order.
  */
 #ifndef EP_H_
 #define EP_H_
@@ -364,14 +367,13 @@ ep_status_t ep_map_replicas(const void *idx, int idx_is_int64, int T, int k,
  * begins.
  *
  * Sharing: every call on a device uses the same array, which keeps the
- * last call's contents (it is zero-filled when the module loads).  Each
- * call clears the part that must start at zero (the 16-byte ticket) with
- * a 16-byte cudaMemsetAsync on `stream` before its kernels run: a call
- * that completes leaves the ticket at zero anyway, but one that raced
- * with another might not, and the clear keeps that from spoiling later
- * calls.  Calls whose work overlaps on the GPU (different streams, no
- * ordering between them) race on the array and give wrong layouts: order
- * them on one stream, or use ep_get_layout with one workspace per stream.
+ * last call's contents (it is zero-filled when the module loads).  The
+ * only part that must start at zero, the 16-byte ticket, is left at zero
+ * by every call's own kernels, even after calls that overlapped; nothing
+ * else is enqueued.  Calls whose work overlaps on the GPU (different
+ * streams, no ordering between them) race on the array and give wrong
+ * layouts: order them on one stream, or use ep_get_layout with one
+ * workspace per stream.
  */
 ep_status_t ep_get_layout_noalloc(const void *idx, int idx_is_int64, int T,
                                   int k, int E, int R, int32_t *cnt_e,
