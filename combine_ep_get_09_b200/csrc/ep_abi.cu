@@ -159,7 +159,7 @@ cudaError_t raise_dynamic_smem(const void *kernel, int bytes) {
 
 extern "C" {
 
-int ep_abi_version(void) { return 4; }
+int ep_abi_version(void) { return 5; }
 
 const char *ep_last_error_string(void) { return g_err; }
 

@@ -66,7 +66,11 @@ struct Params {
   unsigned *ticket;  // tiled path
   int32_t *cols;     // tiled path: [ntiles][E + R]
   int tile_T, ntiles;
-  int stage;         // cluster path: the CTA's checked ids live in shared memory
+  int stage;         // cluster / grid path: the CTA's checked ids live in shared memory
+  unsigned *gbar;    // grid path: arrivals at barrier 1, at barrier 2, departures
+  int first_polls;   // grid path: poll limit of the first barrier's wait
+  int32_t *gcols;    // grid path: [E + R][CTAs] per-CTA counts, then their prefixes
+  int32_t *gtot;     // grid path: [E + R] totals
 };
 
 // Expert id from a raw id value: -1 for a dropped or bad slot (a bad one
@@ -529,6 +533,154 @@ __global__ void __launch_bounds__(kThreads, 1) layout_cluster_kernel(Params p) {
     p.recv_src[r] = -1;
 }
 
+// ------------------------------------------------------------- grid path
+//
+// Mid-size batches on every SM instead of one cluster's 16: one CTA of
+// kGridThreads per SM, launched cooperatively so that all of them run at
+// once, each ranking a contiguous token range as a cluster CTA does.  The
+// per-CTA counts meet in the workspace: after a first grid barrier, CTA c
+// scans columns c, c + G, ... of the [E + R][G] count matrix over the CTAs
+// (exclusive, in place) and writes their totals; after a second barrier
+// every CTA reads its own prefixes and the totals and places its slots.
+// Both barriers are bounded waits (EP_ERR_TIMEOUT in d_err when one gives
+// up); the last CTA to leave sets the barrier counters back to zero.
+constexpr int kGridThreads = 512;
+constexpr int kGridMaxCtas = 160;               // the workspace is sized for this many
+constexpr size_t kGridHeaderBytes = 16;            // three counters, padded
+constexpr size_t kGridMaxWsBytes = 256u << 10;     // larger E + R: the cluster kernel
+constexpr int kMaxGridPolls = 1 << 20;             // x ~0.1 us of sleep each
+
+// Arrive at the grid barrier counter `ctr` and wait, polling at most
+// `max_polls` times, until all `n_ctas` CTAs have; false when the wait gave
+// up.  Every thread of every CTA must call it.
+__device__ bool grid_sync(unsigned *ctr, unsigned n_ctas, int max_polls, int *s_ok) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's writes before its arrival
+    atomicAdd(ctr, 1u);
+    int ok = 1;
+    for (int polls = 0; *reinterpret_cast<volatile unsigned *>(ctr) < n_ctas; ++polls) {
+      if (polls >= max_polls) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(100);
+    }
+    __threadfence();  // the other CTAs' writes after their arrivals
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
+int grid_smem_bytes(int E, int R, long staged) {
+  return ((kGridThreads / kWarp) * (E + R + 1) + 2 * (E + R)) * static_cast<int>(sizeof(int)) +
+         static_cast<int>(((staged * 2 + 15) / 16) * 16);
+}
+
+template <typename IdT>
+__global__ void __launch_bounds__(kGridThreads, 1) layout_grid_kernel(Params p) {
+  extern __shared__ int smem[];
+  const int E = p.E, R = p.R, C = E + R, ld = hist_ld(p);
+  const int tid = threadIdx.x, lane = tid & 31, nt = blockDim.x, w = tid >> 5, nw = nt >> 5;
+  const int G = gridDim.x, cta = blockIdx.x;
+  int *hist = smem;              // [warps][E + R + 1]
+  int *before = hist + nw * ld;  // [C] counts of the lower CTAs
+  int *tot = before + C;         // [C] totals, then exclusive offsets
+  short *ids_smem = reinterpret_cast<short *>(tot + C);  // staged ids
+  __shared__ int wsum[66];
+  __shared__ int s_ok;
+  const IdT *idx = static_cast<const IdT *>(p.idx);
+  const bool stage = p.stage != 0;
+
+  const int t_beg = static_cast<int>(static_cast<long>(p.T) * cta / G);
+  const int t_end = static_cast<int>(static_cast<long>(p.T) * (cta + 1) / G);
+  const long s_beg = static_cast<long>(t_beg) * p.k;
+  const long n = static_cast<long>(t_end - t_beg) * p.k;
+
+  for (int i = tid; i < nw * ld; i += nt) hist[i] = 0;
+  __syncthreads();
+  pdl_wait();
+  long seg_end;
+  const long seg_beg = warp_slice(n, w, nw, &seg_end);
+  SegRanks sr;
+  rank_segment(idx, s_beg + seg_beg, s_beg + seg_end, p, p.d_err, hist + w * ld, p.slot_pos,
+               sr, stage ? ids_smem : nullptr, s_beg);
+  if (stage) __syncthreads();  // every warp's ids are in shared memory
+  rank_mask<IdT>(p, t_beg, t_end, hist + w * ld, stage ? ids_smem : nullptr);
+  __syncthreads();
+  // one thread per column: exclusive prefix over this CTA's warps; the
+  // CTA's count goes to its slot of the column in the workspace
+  for (int col = tid; col < C; col += nt) {
+    int run = 0;
+    for (int v = 0; v < nw; ++v) {
+      const int x = hist[v * ld + col];
+      if (col < E) hist[v * ld + col] = run;
+      run += x;
+    }
+    p.gcols[static_cast<long>(col) * G + cta] = run;
+  }
+  bool ok = grid_sync(&p.gbar[0], G, p.first_polls, &s_ok);
+  if (ok) {
+    // columns cta, cta + G, ...: one warp each, exclusive over the CTAs;
+    // the whole column (G <= kGridMaxCtas values) is loaded before any of
+    // it is scanned, so that it costs one round trip to L2
+    constexpr int kPer = (kGridMaxCtas + 31) / 32;
+    for (int col = cta + G * w; col < C; col += G * nw) {
+      int32_t *colp = p.gcols + static_cast<long>(col) * G;
+      int x[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = 32 * j + lane;
+        x[j] = i < G ? __ldcg(colp + i) : 0;
+      }
+      int carry = 0;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = 32 * j + lane;
+        const int incl = warp_inclusive_scan(x[j]);
+        if (i < G) colp[i] = carry + incl - x[j];
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) p.gtot[col] = carry;
+    }
+  }
+  ok = grid_sync(&p.gbar[1], G, kMaxGridPolls, &s_ok) && ok;
+  if (ok) {
+    for (int col = tid; col < C; col += nt) {
+      before[col] = __ldcg(p.gcols + static_cast<long>(col) * G + cta);
+      tot[col] = __ldcg(p.gtot + col);
+    }
+    __syncthreads();
+    // exclusive scans of the expert totals (their offsets; CTA 0 writes
+    // them with the counts) and of the rank totals
+    const int n_kept = block_scan_counts(
+        tot, nullptr, E, cta == 0 ? p.cnt_e : nullptr, cta == 0 ? p.off_e : nullptr, tot + E,
+        R, cta == 0 ? p.cnt_r : nullptr, cta == 0 ? p.off_r : nullptr, wsum, nullptr);
+    place_segment(idx, s_beg + seg_beg, s_beg + seg_end, p.k, E, hist + w * ld, sr,
+                  p.slot_pos, p.recv_src, before, tot);
+    // rows nobody fills (past the kept ones)
+    const long N = static_cast<long>(p.T) * p.k;
+    for (long r = n_kept + static_cast<long>(cta) * nt + tid; r < N;
+         r += static_cast<long>(G) * nt)
+      p.recv_src[r] = -1;
+  } else if (tid == 0 && p.d_err != nullptr) {
+    atomicExch(reinterpret_cast<int *>(p.d_err), EP_ERR_TIMEOUT);
+  }
+  // every CTA is past both barriers once all have left: the last one out
+  // sets the counters back to zero for the next call on this workspace
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(&p.gbar[2], 1u) == static_cast<unsigned>(G - 1)) {
+      p.gbar[0] = 0u;
+      p.gbar[1] = 0u;
+      p.gbar[2] = 0u;
+      __threadfence();
+    }
+  }
+}
+
 // ------------------------------------------------------------- tiled path
 
 template <typename IdT>
@@ -696,6 +848,28 @@ int tile_tokens(int T) {
 
 bool cluster_path(int T, int k) { return static_cast<long>(T) * k <= kClusterMaxSlots; }
 
+// Batches from this many slots up to kClusterMaxSlots take the grid
+// kernel when its workspace is small enough.  Its fixed cost (about 12 us
+// a launch in CUDA graphs, whatever the size) is above the cluster
+// kernel's below that: 11.7 against 8.8 us at 32768 slots, even at 65536
+// (12.0 / 11.3 warm, 16.2 / 16.9 after a flush), 12.0 against 18.0 at
+// 131072 and 13.9 against 31.9 at 262144.
+constexpr long kGridMinSlots = 65536;
+
+int grid_ctas() { return min(device_sm_count(), kGridMaxCtas); }
+
+// Workspace of the grid kernel, sized for kGridMaxCtas CTAs so that it
+// does not depend on the device.
+size_t grid_ws_bytes(int E, int R) {
+  const size_t C = static_cast<size_t>(E) + R;
+  return kGridHeaderBytes + (C * kGridMaxCtas + C) * sizeof(int32_t);
+}
+
+bool grid_path(int T, int k, int E, int R) {
+  const long N = static_cast<long>(T) * k;
+  return N >= kGridMinSlots && N <= kClusterMaxSlots && grid_ws_bytes(E, R) <= kGridMaxWsBytes;
+}
+
 // Largest cluster (<= 16 CTAs) the device can schedule for this kernel with
 // `smem` bytes per CTA; cached per (device, id type, smem size).
 // Largest cluster (16, else the portable 8) the GPU can run with CTAs of
@@ -774,6 +948,42 @@ cudaError_t launch_cluster(Params p, cudaStream_t s, int *launches) {
   return launch_cluster_with<IdT, kClusterThreads>(p, n_ctas, s, launches);
 }
 
+// The grid kernel: one CTA per SM, launched cooperatively (all CTAs
+// resident at once, or the launch is refused) with programmatic stream
+// serialization.  Returns the launch error; nothing runs when it fails.
+template <typename IdT>
+cudaError_t launch_grid(Params p, int ctas, void *ws, cudaStream_t s) {
+  auto kern = layout_grid_kernel<IdT>;
+  const long per_cta_slots = static_cast<long>((p.T + ctas - 1) / ctas) * p.k;
+  const int smem_max = max_dynamic_smem(reinterpret_cast<const void *>(kern));
+  int smem = grid_smem_bytes(p.E, p.R, 0);
+  p.stage = 0;
+  if (per_cta_slots <= kStageIdsMax && grid_smem_bytes(p.E, p.R, per_cta_slots) <= smem_max) {
+    smem = grid_smem_bytes(p.E, p.R, per_cta_slots);
+    p.stage = 1;
+  }
+  const cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern), smem);
+  if (err != cudaSuccess) return err;
+  p.gbar = static_cast<unsigned *>(ws);
+  // the testing switch of the bounded waits reaches the first barrier too
+  p.first_polls = first_wait_polls() == 0 ? 0 : kMaxGridPolls;
+  p.gcols = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + kGridHeaderBytes);
+  p.gtot = p.gcols + static_cast<long>(p.E + p.R) * ctas;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(kGridThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 template <typename IdT>
 cudaError_t launch_tiled(Params p, cudaStream_t s, int *launches) {
   const int C = p.E + p.R, ld = p.E + p.R + 1;
@@ -797,7 +1007,9 @@ cudaError_t launch_tiled(Params p, cudaStream_t s, int *launches) {
 }  // namespace
 
 size_t layout_workspace_bytes(int T, int k, int E, int R) {
-  if (T <= 0 || cluster_path(T, k)) return 0;
+  if (T <= 0) return 0;
+  if (grid_path(T, k, E, R)) return grid_ws_bytes(E, R);
+  if (cluster_path(T, k)) return 0;
   const int tile_T = tile_tokens(T);
   const long ntiles = (T + tile_T - 1) / tile_T;
   return kTicketBytes + static_cast<size_t>(ntiles) * (E + R) * sizeof(int32_t);
@@ -822,6 +1034,22 @@ cudaError_t launch_layout(const LayoutArgs &a, cudaStream_t s, int *launches) {
   p.recv_src = a.recv_src;
   p.in_rank = a.in_rank;
   p.d_err = a.d_err;
+  if (a.ws != nullptr && grid_path(a.T, a.k, a.E, a.R)) {
+    const int ctas = grid_ctas();
+    cudaError_t err;
+    if (a.id_kind == kIdsMask)
+      err = launch_grid<uint8_t>(p, ctas, a.ws, s);
+    else
+      err = a.id_kind == kIdsInt64 ? launch_grid<int64_t>(p, ctas, a.ws, s)
+                                   : launch_grid<int32_t>(p, ctas, a.ws, s);
+    if (err == cudaSuccess) {
+      ++*launches;
+      return err;
+    }
+    // refused (for instance fewer SMs than CTAs in a green context): the
+    // cluster kernel needs no co-residency beyond its own cluster
+    cudaGetLastError();
+  }
   if (cluster_path(a.T, a.k)) {
     if (a.id_kind == kIdsMask) return launch_cluster<uint8_t>(p, s, launches);
     return a.id_kind == kIdsInt64 ? launch_cluster<int64_t>(p, s, launches)

@@ -71,7 +71,8 @@ typedef int ep_status_t;
 #define EP_MAX_E 1024  /* experts                          */
 #define EP_MAX_R 64    /* logical ranks                    */
 
-/* Version of this ABI (incremented on any signature change): 4. */
+/* Version of this ABI (incremented on any signature change, and when the
+ * workspace a call needs changes): 5. */
 int ep_abi_version(void);
 
 /* Message of the last error returned on this host thread ("" if none). */
@@ -82,7 +83,14 @@ uint64_t ep_kernel_launches(void);
 
 /*
  * Bytes of device workspace ep_get_layout needs for (T, k, E, R); 0 when the
- * single-block path applies (then ws may be NULL).
+ * single-CTA or cluster kernel applies (then ws may be NULL).  The kernel
+ * depends on the slots T*k: up to 2048 one CTA; below 65536 one cluster of
+ * up to 16 CTAs; from 65536 to 2^19 one CTA on each SM (a cooperative
+ * launch; workspace: 16 bytes of barrier counters plus (E + R) * 161 int32
+ * counts), unless that workspace would exceed 256 KiB, when the cluster
+ * again; above 2^19 the tiled pair (16 bytes plus one row of E + R counts
+ * per tile).  A launch refused for co-residency (for instance fewer free
+ * SMs than CTAs in a green context) falls back to the cluster kernel.
  */
 size_t ep_layout_workspace_bytes(int T, int k, int E, int R);
 
@@ -115,7 +123,8 @@ size_t ep_layout_workspace_bytes(int T, int k, int E, int R);
  * Outputs: int32 arrays 4-byte aligned, in_rank 1-byte aligned.
  * ws, ws_bytes  device scratch of at least ep_layout_workspace_bytes()
  *              bytes, 16-byte aligned.  It must be zero-filled before its
- *              first use; every call leaves it zero-filled again, so one
+ *              first use; every call leaves its counters (the first 16
+ *              bytes) at zero again and overwrites the rest, so one
  *              buffer serves a sequence of stream-ordered calls (not
  *              concurrent ones).
  * d_err        optional (may be NULL) device int32; set to EP_ERR_INDEX when
@@ -181,7 +190,7 @@ ep_status_t ep_dispatch(const void *x, int T, int H, int k,
  * tells which ran).
  *
  * idx .. recv_src, ws, ws_bytes: as ep_get_layout (ws is needed only when
- * ep_layout_workspace_bytes(T, k, E, R) > 0, i.e. for T*k > 2^19).
+ * ep_layout_workspace_bytes(T, k, E, R) > 0, i.e. for T*k >= 65536).
  * x, H, fp8, recv, recv_scale, num_sms: as ep_dispatch.
  * d_err receives EP_ERR_INDEX for a bad id and EP_ERR_TIMEOUT as in
  * ep_dispatch.  All argument checks of both calls apply, before anything
@@ -292,7 +301,7 @@ ep_status_t ep_pad_layout(const int32_t *cnt_e, const int32_t *slot_pos,
  * in_rank   [T,R] uint8 (0 / nonzero), rank_row [T,R] int32,
  * rank_src  [T*R] int32, cnt_r [R], off_r [R+1] int32.
  * T >= 0, 1 <= R <= EP_MAX_R, T*R < 2^31.  ws / ws_bytes as ep_get_layout,
- * sized by ep_rank_layout_workspace_bytes (0 for T*R <= 2^19).
+ * sized by ep_rank_layout_workspace_bytes (0 for T*R < 65536).
  */
 size_t ep_rank_layout_workspace_bytes(int T, int R);
 ep_status_t ep_get_rank_layout(const uint8_t *in_rank, int T, int R,
@@ -394,8 +403,14 @@ ep_status_t ep_get_layout_noalloc(const void *idx, int idx_is_int64, int T,
  * incomplete.  With on != 0, the first such wait of every CTA of kernels
  * launched afterwards gives up at once, without polling, while its copy
  * still lands normally -- so that path can be run and checked without
- * making any copy fail.  on == 0 (the default) restores the normal limit.
- * Process-wide; for tests only (the pages have no counterpart).
+ * making any copy fail.  The grid layout kernel (ep_get_layout for
+ * 65536 <= T*k <= 2^19) waits the same way, bounded, at two barriers
+ * between its CTAs; the switch makes the first of them give up at once in
+ * every CTA that has not seen all CTAs arrive: such a CTA records
+ * EP_ERR_TIMEOUT and places none of its slots, and the workspace's
+ * counters are still left at zero.  on == 0 (the default) restores the
+ * normal limits.  Process-wide; for tests only (the pages have no
+ * counterpart).
  */
 void ep_debug_expire_first_wait(int on);
 

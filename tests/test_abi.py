@@ -29,17 +29,24 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version():
-    assert ep.lib().ep_abi_version() == 4
+    assert ep.lib().ep_abi_version() == 5
 
 
 def test_workspace_sizes():
-    # the cluster path (T*k <= 2^19) needs none; the tiled path one row of
-    # E + R counts per tile (at most 296 tiles of >= 128 tokens) plus a
+    # the single-CTA and cluster paths (T*k < 65536) need none; the grid
+    # path (65536 <= T*k <= 2^19) three 4-byte barrier counters padded to 16
+    # bytes plus an [E + R][160] count matrix and E + R totals, when that is
+    # at most 256 KiB (else the cluster path again); the tiled path one row
+    # of E + R counts per tile (at most 296 tiles of >= 128 tokens) plus a
     # 16-byte ticket
     assert ep.ep_layout_workspace_bytes(128, 8, 256, 8) == 0
     assert ep.ep_layout_workspace_bytes(0, 8, 256, 8) == 0
     assert ep.ep_layout_workspace_bytes(4096, 8, 256, 8) == 0
-    assert ep.ep_layout_workspace_bytes(65536, 8, 256, 8) == 0
+    assert ep.ep_layout_workspace_bytes(8191, 8, 256, 8) == 0
+    assert ep.ep_layout_workspace_bytes(8192, 8, 256, 8) == 16 + (264 * 160 + 264) * 4
+    assert ep.ep_layout_workspace_bytes(65536, 8, 256, 8) == 16 + (264 * 160 + 264) * 4
+    assert ep.ep_layout_workspace_bytes(32768, 8, 128, 16) == 16 + (144 * 160 + 144) * 4
+    assert ep.ep_layout_workspace_bytes(32768, 8, 1024, 64) == 0   # 696 KiB: cluster path
     assert ep.ep_layout_workspace_bytes(65537, 8, 256, 8) == 16 + 296 * 264 * 4
     assert ep.ep_layout_workspace_bytes(70000, 8, 128, 16) == 16 + 296 * 144 * 4
     assert ep.ep_layout_workspace_bytes(300000, 2, 16, 16) == 16 + 296 * 32 * 4

@@ -114,6 +114,26 @@ def test_layout_workspace_reused_across_calls():
     assert int(ws[:4].view(torch.int32).item()) == 0   # ticket back at 0
 
 
+def test_layout_grid_workspace_reused_across_calls():
+    # grid path (one CTA per SM, 65536 <= T*k <= 2^19): the barrier counters
+    # in the workspace go back to zero, so one zeroed buffer serves many
+    # calls in stream order
+    cfg = workloads.CONFIGS["large"]
+    ws = torch.zeros(ep.ep_layout_workspace_bytes(cfg.T, cfg.k, cfg.E, cfg.R),
+                     dtype=torch.uint8, device="cuda")
+    assert ws.numel() > 0
+    for seed, T in ((0, cfg.T), (1, 9000), (2, 20000)):
+        assert 65536 <= T * cfg.k <= 1 << 19
+        b = workloads.make_batch(cfg, seed, T=T, H=8, drop_frac=0.05, dup_frac=0.05)
+        d_err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        L = ep.ep_get_layout(b.idx.cuda(), cfg.E, cfg.R, ws=ws, d_err=d_err)
+        host = {key: getattr(L, key).cpu().numpy() for key in
+                ("cnt_e", "cnt_r", "in_rank", "off_e", "off_r", "slot_pos", "recv_src")}
+        host["status"] = ep.ep_read_error(d_err)
+        assert_layout_equal(host, oracle.layout(b.idx, cfg.E, cfg.R))
+        assert not ws[:12].view(torch.int32).any()    # counters back at 0
+
+
 # ---------------------------------------------------------------- dispatch
 
 def _dispatch_bf16_check(cfg, b, num_sms=0):

@@ -134,3 +134,23 @@ def test_fused_layout_dispatch_wait_times_out_then_recovers(num_sms, fp8):
     else:
         want = oracle.dispatch_bf16(b.x, ref["slot_pos"], T * k)
         np.testing.assert_array_equal(tensor_bits16(recv), want)
+
+
+def test_grid_layout_barrier_times_out_then_recovers():
+    # the grid layout kernel (one CTA per SM) meets at two barriers between
+    # its CTAs; the switch makes the first give up in every CTA that has not
+    # seen all arrive, and the workspace's counters must still be left at 0
+    cfg = workloads.CONFIGS["large"]
+    b = workloads.make_batch(cfg, 35, H=8)
+    idx = b.idx.cuda()
+    ws = torch.zeros(ep.ep_layout_workspace_bytes(b.T, cfg.k, cfg.E, cfg.R),
+                     dtype=torch.uint8, device="cuda")
+    out = ep.empty_layout(b.T, cfg.k, cfg.E, cfg.R, "cuda")
+    call = lambda e: ep.ep_get_layout(idx, cfg.E, cfg.R, out=out, ws=ws, d_err=e)  # noqa: E731
+    assert _expired(call) == ep.EP_ERR_TIMEOUT
+    assert not ws[:12].view(torch.int32).any()
+    _normal(call)
+    ref = oracle.layout(b.idx, cfg.E, cfg.R)
+    host = {key: getattr(out, key).cpu().numpy() for key in ref if key != "status"}
+    host["status"] = ref["status"]
+    assert_layout_equal(host, ref)

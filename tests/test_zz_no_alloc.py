@@ -46,9 +46,11 @@ def _check_against(got, want: dict, name: str):
                                       err_msg=f"{name}: {key}")
 
 
-# two batches of the large workload's routing (128 experts in 16 ranks,
-# top-8) big enough for the tiled layout, the one that uses the scratch
-BATCHES = ((70000, 0), (66000, 1))
+# batches of the large workload's routing (128 experts in 16 ranks, top-8)
+# whose layouts use the scratch: two for the tiled kernels (T*k > 2^19),
+# then one for the grid kernel (65536 <= T*k <= 2^19, barrier counters
+# in the scratch), after a tiled one on the same array
+BATCHES = ((70000, 0), (66000, 1), (32768, 2))
 
 
 @pytest.mark.gpu
