@@ -48,13 +48,14 @@ def test_layout_full_size(name, seed):
     assert_layout_equal(g, oracle.layout(b.idx, cfg.E, cfg.R))
 
 
-@pytest.mark.parametrize("T", [0, 1, 3, 31, 127, 512, 513, 2047, 4097, 9999, 32769,
-                               65536, 65537, 70001])
+@pytest.mark.parametrize("T", [0, 1, 3, 31, 127, 512, 513, 2047, 4097, 8191, 8192, 9999,
+                               32769, 65536, 65537, 70001])
 @pytest.mark.parametrize("int32_ids", [False, True])
 def test_layout_ragged_and_both_id_types(T, int32_ids):
-    # k = 8: up to T = 512 one CTA, then a cluster of up to 16 CTAs (4096
-    # slots each, so 32769 is the first 16-CTA batch); T*k = 2^19
-    # (T = 65536) is the largest cluster case, 65537 the first tiled one
+    # k = 8: up to T = 256 one CTA, then a cluster of up to 16 CTAs (512 or
+    # 1024 threads) up to 65535 slots (T = 8191); from T = 8192 (65536
+    # slots) one CTA per SM with grid barriers; T*k = 2^19 (T = 65536) is
+    # the largest such case, 65537 the first tiled one
     cfg, b = _batch("prefill", 3, T=T, H=8, drop_frac=0.1, dup_frac=0.1)
     _, g = gpu_layout(b.idx, cfg.E, cfg.R, int32_ids=int32_ids)
     assert_layout_equal(g, oracle.layout(b.idx, cfg.E, cfg.R))
@@ -63,8 +64,12 @@ def test_layout_ragged_and_both_id_types(T, int32_ids):
 @pytest.mark.parametrize("T,k,E,R", [(500, 1, 1, 1), (300, 32, 64, 64),
                                      (2500, 32, 1024, 64), (4000, 4, 1024, 1),
                                      (100000, 2, 16, 16), (300000, 2, 16, 16),
-                                     (20000, 32, 1024, 64)])
+                                     (20000, 32, 1024, 64), (9000, 8, 1024, 64),
+                                     (70000, 1, 2, 2)])
 def test_layout_extreme_shapes(T, k, E, R):
+    # (9000, 8, 1024, 64): a grid-path size whose count matrix would exceed
+    # 256 KiB, so the cluster kernel runs; (70000, 1, 2, 2): the grid path
+    # with a 4-column count matrix and a single slot per token
     rng = np.random.default_rng(T + k + E)
     idx = np.argsort(rng.random((T, E)), axis=1)[:, :k] if E <= 64 else \
         np.stack([rng.choice(E, k, replace=False) for _ in range(T)])

@@ -45,9 +45,10 @@ def test_rank_layout_workloads(name):
     np.testing.assert_array_equal(RL.cnt_r.cpu().numpy(), L.cnt_r.cpu().numpy())
 
 
-@pytest.mark.parametrize("T", [0, 1, 255, 2049, 70001])
+@pytest.mark.parametrize("T", [0, 1, 255, 2049, 8192, 65536, 70001])
 def test_rank_layout_ragged_and_tiled(T):
-    # T * R above 2^19 (70001 x 8) takes the tiled layout with a workspace
+    # T * R from 65536 (8192 x 8) to 2^19 (65536 x 8) takes the grid
+    # kernel, above 2^19 (70001 x 8) the tiled layout, both with a workspace
     cfg, b, L = _mask("prefill", 1, T=T, drop=0.2)
     _check_rank_layout(L.in_rank)
 
