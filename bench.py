@@ -14,15 +14,19 @@ HBM, so no step pays for write-backs that are not its own.
 
 Prints one JSON line.  ``value`` is algorithmic HBM bytes moved per second
 over all ranks (each source byte read once, each destination byte written
-once); ``roofline`` is the dominant kernel against the measured copy
-bandwidth; ``decode`` is the 128-token decode workload in microseconds per
-call (layout + FP8 dispatch + combine), unfused and with the fused
-layout + dispatch kernel, plain and in CUDA graphs; ``rank_dedup``,
+once), the steps timed with events at their ends only; ``kernels`` and
+``instrumented_step`` come from the same steps with events around every
+kernel; ``roofline`` is the combine (the longest kernel) against the
+measured copy bandwidth, timed live in the timed steps; ``decode`` is the
+128-token decode workload in microseconds per call (layout + FP8 dispatch +
+combine), unfused and with the fused layout + dispatch kernel, warm in
+CUDA graphs of 20 calls and after an L2 flush; ``rank_dedup``,
 ``combine_variants`` (aligned layout, FP8 combine, expert replicas) and
 ``sm_budget_overlap`` (copy kernels beside a GEMM, with and without a
 green-context SM partition) measure the further forms of the path;
-``cpu_baseline`` times the CPU oracle on a bounded sample; ``e2e`` runs the
-same step from pinned host buffers with the copies inside the timed region.
+``cpu_baseline`` times the CPU oracle on whole steps of the same batch;
+``e2e`` runs the same step from pinned host buffers with the copies inside
+the timed region; ``summary`` repeats the headline figures at the end.
 
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no
 data-path collective); times are the max over ranks.

@@ -2,14 +2,17 @@
 // counts, the token-in-rank mask, exclusive prefix offsets and the stable
 // receive row of every (token, slot).
 //
-// Two paths, both deterministic (no ordering ever depends on atomics) and
-// neither with a CTA that waits on another through memory:
-//  * cluster (T*k <= kClusterMaxSlots): one launch of a thread-block
+// Three paths, all deterministic (no ordering ever depends on atomics):
+//  * cluster (T*k below kGridMinSlots): one launch of a thread-block
 //    cluster of up to 16 CTAs (a single plain CTA for small batches such as
 //    a 128-token decode step).  Each CTA ranks its contiguous token range,
 //    the CTAs exchange their per-expert counts through distributed shared
 //    memory between two hardware cluster barriers, and every CTA then
 //    places its own slots.  No global workspace.
+//  * grid (kGridMinSlots <= T*k <= kClusterMaxSlots): the same per-CTA work
+//    on one CTA per SM, launched cooperatively; the counts meet in the
+//    caller's workspace between two grid barriers, the only waits of one
+//    CTA on others in this library, each bounded.
 //  * tiled (larger batches): a counting kernel writes one histogram row per
 //    tile of tokens to the caller's workspace, and the last tile to finish
 //    (ticket taken with atomicInc, which wraps it back to 0) turns the rows
