@@ -15,8 +15,10 @@
 //    kStages items ahead; every thread then folds its 16 bytes of the k
 //    rows and writes one 16-byte vector of the output.  The bytes in flight
 //    live in shared memory, not registers, which keeps HBM busy on this
-//    read-dominated gather.  Chunks of 256 vectors, or 64 when each item
-//    then still gets a CTA of its own in one wave (small batches).
+//    read-dominated gather.  Chunks of 256 vectors.
+//  * combine_item_kernel (k <= 8, when every item of 64-vector chunks gets
+//    a CTA of its own in one wave, e.g. a decode batch): one item per CTA,
+//    the k rows' vectors loaded straight into registers.
 //  * combine_reg_kernel (any k <= 32): a warp per item with 128-bit loads
 //    of 8 slot rows at a time into registers.
 //  * combine_fp8_bulk_kernel / combine_fp8_reg_kernel: the same for expert
@@ -38,12 +40,11 @@ constexpr int kBulkMaxK = 8;     // slot rows one bulk stage holds
 // shape (alone: 77.8 us with 2 stages of 4 KB chunks, 82.0 with 3 stages
 // of 2 KB, 88.1 with 3 of 4 KB, 141 with one CTA per SM and 6 stages).
 constexpr int kStages = 2;
-// 16-byte vectors per row chunk (= threads of the bulk kernel): 256 in
-// general; 64 when every item of the smaller chunks still gets a CTA of its
-// own in one wave (a decode batch), which shortens each CTA's chain.  (128
-// fits one wave only where 64 does too: 6 of its CTAs fit an SM, 13 of 64's.)
+// 16-byte vectors per row chunk (= threads of the bulk kernel): 256; the
+// small-batch kernel takes items of 64 vectors.
 constexpr int kChunkVec = 256;
 constexpr int kSmallChunkVec = 64;
+constexpr int kSmallItemCtasPerSm = 13;
 template <int CHV>
 constexpr int bulk_smem() { return kStages * kBulkMaxK * CHV * 16; }
 
@@ -157,6 +158,42 @@ __global__ void __launch_bounds__(kChunkVec)
     for (long q = i; q < min(n_mine, i + kStages); ++q)
       mbar_wait_bounded(&full[q % kStages], static_cast<unsigned>((q / kStages) & 1));
   }
+}
+
+// One CTA of kSmallChunkVec threads per (token, chunk of kSmallChunkVec
+// 16-byte vectors), for batches whose items all get a CTA in one wave: the
+// slot rows and weights are read by every thread (broadcast loads), then
+// each thread loads its vector of the k rows straight into registers, so
+// the CTA's chain is two round trips with no shared memory or barrier.
+__global__ void __launch_bounds__(kSmallChunkVec)
+    combine_item_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
+                        const int32_t *__restrict__ slot_pos, const float *__restrict__ w,
+                        uint4 *__restrict__ out, long n_rows) {
+  const int nchunks = (Hv + kSmallChunkVec - 1) / kSmallChunkVec;
+  const int t = blockIdx.x / nchunks;
+  const int v = (blockIdx.x - t * nchunks) * kSmallChunkVec + threadIdx.x;
+  pdl_wait();
+  const long tk = static_cast<long>(t) * k;
+  int row[kBulkMaxK];
+  float wj[kBulkMaxK];
+#pragma unroll
+  for (int j = 0; j < kBulkMaxK; ++j) {
+    row[j] = j < k ? __ldg(slot_pos + tk + j) : -1;
+    wj[j] = j < k ? (w != nullptr ? __ldg(w + tk + j) : 1.0f) : 0.0f;
+  }
+  if (v >= Hv) return;
+  uint4 val[kBulkMaxK];
+#pragma unroll
+  for (int j = 0; j < kBulkMaxK; ++j)
+    val[j] = row[j] >= 0 && row[j] < n_rows ? ld_stream_v4(y + static_cast<long>(row[j]) * Hv + v)
+                                            : make_uint4(0, 0, 0, 0);
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kBulkMaxK; ++j)
+    if (row[j] >= 0 && row[j] < n_rows) fma_bf16x8(acc, wj[j], val[j]);  // dropped: nothing
+  st_stream_v4(out + static_cast<long>(t) * Hv + v, to_bf16x8(acc));
 }
 
 __global__ void __launch_bounds__(kRegThreads, 2)
@@ -418,12 +455,20 @@ cudaError_t launch_combine(const void *y, long n_rows, int T, int H, int k,
                         static_cast<uint4 *>(out), n_rows, first_wait_polls(), d_err);
     };
     if (T == 0) return cudaSuccess;
-    {  // small chunks when each of their items gets a CTA in one wave
-      auto kern = combine_bulk_kernel<kSmallChunkVec>;
+    {  // small batches: one item of 64 vectors per CTA, loaded straight into
+       // registers (decode combine 3.59 -> 2.88 us a call in graphs of 20,
+       // against the bulk-copy pipeline with 1 KB chunks), while the items
+       // fit kSmallItemCtasPerSm CTAs per SM (the bound under which it was
+       // measured)
       const long items = static_cast<long>(T) * ((Hv + kSmallChunkVec - 1) / kSmallChunkVec);
-      const long cap = persistent_grid(reinterpret_cast<const void *>(kern), kSmallChunkVec,
-                                       bulk_smem<kSmallChunkVec>(), 1L << 40, num_sms);
-      if (items <= cap) return launch(kern, kSmallChunkVec, items, items);
+      const long cap = static_cast<long>(num_sms > 0 ? num_sms : device_sm_count()) *
+                       kSmallItemCtasPerSm;
+      if (items <= cap) {
+        ++*launches;
+        return launch_pdl(combine_item_kernel, dim3(items), dim3(kSmallChunkVec), 0, s, 1,
+                          static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,
+                          static_cast<uint4 *>(out), n_rows);
+      }
     }
     auto kern = combine_bulk_kernel<kChunkVec>;
     constexpr int smem = bulk_smem<kChunkVec>();
