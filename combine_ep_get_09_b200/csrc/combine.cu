@@ -6,19 +6,24 @@
 // All kernels here run the same fp32 fma chain in slot order, so their
 // results are bit-identical to one another:
 //
-//  * combine_bulk_kernel<chunk> (k <= 8, the common case): a bulk-copy
-//    (TMA) pipeline.  A CTA of `chunk` threads walks a contiguous range of
-//    work items (token t, chunk c of 16-byte vectors), the ranges of all
-//    CTAs equal to within one item.  Lanes 0..k-1 of warp 0 read the
-//    token's slot rows and weights and each gathers its row's chunk into
-//    shared memory with cp.async.bulk (completing on the stage's mbarrier),
-//    kStages items ahead; every thread then folds its 16 bytes of the k
-//    rows and writes one 16-byte vector of the output.  The bytes in flight
-//    live in shared memory, not registers, which keeps HBM busy on this
-//    read-dominated gather.  Chunks of 256 vectors.
-//  * combine_item_kernel (k <= 8, when every item of 64-vector chunks gets
-//    a CTA of its own in one wave, e.g. a decode batch): one item per CTA,
-//    the k rows' vectors loaded straight into registers.
+//  * combine_item_kernel (k <= 8; every batch on all SMs): one work item
+//    (token t, chunk of 64 16-byte vectors) per CTA of 64 threads.  Every
+//    thread reads the token's slot rows and weights (broadcast loads),
+//    then its vector of the k rows straight into registers, folds them and
+//    writes one vector of the output.  The grid holds every item, so waves
+//    of CTAs follow one another as SMs free up; measured against the
+//    persistent bulk-copy pipeline below, 96.5 -> 88.1 us inside the
+//    prefill step (73 -> 70 us alone) and 3.59 -> 2.88 us a decode call.
+//  * combine_bulk_kernel<256> (k <= 8 under an SM budget, num_sms > 0, once
+//    the items no longer fit kSmallItemCtasPerSm CTAs per budgeted SM): a
+//    bulk-copy (TMA) pipeline on a persistent grid sized to the budget.  A
+//    CTA of 256 threads walks a contiguous range of (token, 256-vector
+//    chunk) items, the ranges of all CTAs equal to within one item.  Lanes
+//    0..k-1 of warp 0 read the token's slot rows and weights and each
+//    gathers its row's chunk into shared memory with cp.async.bulk
+//    (completing on the stage's mbarrier), kStages items ahead; every
+//    thread then folds its 16 bytes of the k rows and writes one 16-byte
+//    vector of the output.
 //  * combine_reg_kernel (any k <= 32): a warp per item with 128-bit loads
 //    of 8 slot rows at a time into registers.
 //  * combine_fp8_bulk_kernel / combine_fp8_reg_kernel: the same for expert
@@ -41,10 +46,12 @@ constexpr int kBulkMaxK = 8;     // slot rows one bulk stage holds
 // of 2 KB, 88.1 with 3 of 4 KB, 141 with one CTA per SM and 6 stages).
 constexpr int kStages = 2;
 // 16-byte vectors per row chunk (= threads of the bulk kernel): 256; the
-// small-batch kernel takes items of 64 vectors.
+// item kernel takes items of 64 vectors (128 and 256 measured 0.5-3 us
+// slower at the prefill shape).
 constexpr int kChunkVec = 256;
 constexpr int kSmallChunkVec = 64;
 constexpr int kSmallItemCtasPerSm = 13;
+constexpr long kMaxGridX = 2147483647;  // largest gridDim.x
 template <int CHV>
 constexpr int bulk_smem() { return kStages * kBulkMaxK * CHV * 16; }
 
@@ -161,10 +168,10 @@ __global__ void __launch_bounds__(kChunkVec)
 }
 
 // One CTA of kSmallChunkVec threads per (token, chunk of kSmallChunkVec
-// 16-byte vectors), for batches whose items all get a CTA in one wave: the
-// slot rows and weights are read by every thread (broadcast loads), then
-// each thread loads its vector of the k rows straight into registers, so
-// the CTA's chain is two round trips with no shared memory or barrier.
+// 16-byte vectors): the slot rows and weights are read by every thread
+// (broadcast loads), then each thread loads its vector of the k rows
+// straight into registers, so the CTA's chain is two round trips with no
+// shared memory or barrier.  Launched with one CTA per item.
 __global__ void __launch_bounds__(kSmallChunkVec)
     combine_item_kernel(const uint4 *__restrict__ y, int T, int Hv, int k,
                         const int32_t *__restrict__ slot_pos, const float *__restrict__ w,
@@ -455,15 +462,15 @@ cudaError_t launch_combine(const void *y, long n_rows, int T, int H, int k,
                         static_cast<uint4 *>(out), n_rows, first_wait_polls(), d_err);
     };
     if (T == 0) return cudaSuccess;
-    {  // small batches: one item of 64 vectors per CTA, loaded straight into
-       // registers (decode combine 3.59 -> 2.88 us a call in graphs of 20,
-       // against the bulk-copy pipeline with 1 KB chunks), while the items
-       // fit kSmallItemCtasPerSm CTAs per SM (the bound under which it was
-       // measured)
+    {  // one CTA per item of 64 vectors, loaded straight into registers: on
+       // all SMs at any size; under an SM budget only while the items fit
+       // kSmallItemCtasPerSm CTAs per budgeted SM (a grid of more CTAs
+       // would spread over every SM)
       const long items = static_cast<long>(T) * ((Hv + kSmallChunkVec - 1) / kSmallChunkVec);
-      const long cap = static_cast<long>(num_sms > 0 ? num_sms : device_sm_count()) *
-                       kSmallItemCtasPerSm;
-      if (items <= cap) {
+      const bool fits = num_sms > 0
+                            ? items <= static_cast<long>(num_sms) * kSmallItemCtasPerSm
+                            : items <= kMaxGridX;
+      if (fits) {
         ++*launches;
         return launch_pdl(combine_item_kernel, dim3(items), dim3(kSmallChunkVec), 0, s, 1,
                           static_cast<const uint4 *>(y), T, Hv, k, slot_pos, w,

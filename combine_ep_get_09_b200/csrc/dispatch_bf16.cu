@@ -1,12 +1,19 @@
 // dispatch_bf16.cu -- token rows to expert-contiguous receive rows (bf16).
 //
-// A persistent grid-stride loop over work items (token t, chunk c of its
-// row).  A warp loads the chunk once with 128-bit read-only streaming
-// loads, then writes it to each of the token's k receive rows with
-// coalesced streaming stores, so HBM sees each source byte read once and
-// each destination byte written once.  The slot rows of the token are
+// A grid-stride loop over work items (token t, chunk c of its row), one
+// warp per item.  A warp loads the chunk once with 128-bit read-only
+// streaming loads, then writes it to each of the token's k receive rows
+// with coalesced streaming stores, so HBM sees each source byte read once
+// and each destination byte written once.  The slot rows of the token are
 // fetched by lanes 0..k-1 and broadcast with shuffles.  Before waiting on
 // the previous kernel, every warp asks L2 for the x chunks it will copy.
+//
+// On all SMs the grid holds one warp per item, so waves of CTAs follow one
+// another as SMs free up (measured against a persistent grid of 8 CTAs per
+// SM: 91 -> 84 us inside the prefill step); under an SM budget
+// (num_sms > 0) the grid is persistent, sized to the budget.
+#include <algorithm>
+
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -81,8 +88,12 @@ cudaError_t launch_dispatch_bf16(const void *x, int T, int H, int k,
   const long items = static_cast<long>(T) * nchunks;
   if (items == 0) return cudaSuccess;
   auto kern = dispatch_bf16_kernel<kBf16Vec>;
+  constexpr long kWarpsPerCta = kThreads / 32;
+  constexpr long kMaxGridX = 2147483647;
   const long grid =
-      persistent_grid(reinterpret_cast<const void *>(kern), kThreads, 0, items, num_sms);
+      num_sms > 0
+          ? persistent_grid(reinterpret_cast<const void *>(kern), kThreads, 0, items, num_sms)
+          : std::min((items + kWarpsPerCta - 1) / kWarpsPerCta, kMaxGridX);
   ++*launches;
   return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, s, 1, static_cast<const uint4 *>(x), T,
                     Hv, k, slot_pos, static_cast<uint4 *>(recv), n_rows);

@@ -394,11 +394,12 @@ ep_status_t ep_get_layout_noalloc(const void *idx, int idx_is_int64, int T,
 /*
  * ep_debug_expire_first_wait -- testing switch for the bounded waits.
  *
- * The bulk-copy kernels (ep_combine with k <= 8 above the small batches
- * whose (token, 1 KB) items fit 13 CTAs per SM, ep_combine_fp8 with k <= 8,
- * the FP8 ep_dispatch for H % 512 == 0, and both kernels of
- * ep_layout_dispatch) wait for their own asynchronous copies on shared-
- * memory barriers, each wait bounded by an iteration limit; when a limit
+ * The bulk-copy kernels (ep_combine with k <= 8 under an SM budget,
+ * num_sms > 0, once its (token, 1 KB) items no longer fit 13 CTAs per
+ * budgeted SM; ep_combine_fp8 with k <= 8; the FP8 ep_dispatch for
+ * H % 512 == 0; both kernels of ep_layout_dispatch) wait for their own
+ * asynchronous copies on shared-memory barriers, each wait bounded by an
+ * iteration limit; when a limit
  * runs out the kernel records EP_ERR_TIMEOUT in d_err, waits (bounded) for
  * the copies it still has in flight and returns, leaving its output
  * incomplete.  With on != 0, the first such wait of every CTA of kernels

@@ -320,9 +320,11 @@ def test_combine_ragged_hidden_and_drops(H):
     assert _combine_check(cfg, b) == 1.0
 
 
-@pytest.mark.parametrize("num_sms", [1, 29])
-def test_combine_sm_budget(num_sms):
-    cfg, b = _batch("prefill", 3, T=300)
+# under a budget the register kernel runs while its items fit one wave on
+# the budgeted SMs (T = 16 on 29 SMs), the bulk-copy pipeline above that
+@pytest.mark.parametrize("T,num_sms", [(300, 1), (300, 29), (16, 29)])
+def test_combine_sm_budget(T, num_sms):
+    cfg, b = _batch("prefill", 3, T=T)
     assert _combine_check(cfg, b, num_sms=num_sms) == 1.0
 
 

@@ -56,15 +56,16 @@ def _setup(name, seed, T, H):
     return cfg, b, L, ref
 
 
-# the bulk-copy pipeline: T = 200, one 4 KB item per CTA; T = 3000, CTAs
-# walking several items each (small batches, such as 128 tokens, take a
-# kernel with no asynchronous copies to wait for)
-@pytest.mark.parametrize("T", [200, 3000])
-def test_combine_wait_times_out_then_recovers(T):
+# the bf16 combine's bulk-copy pipeline runs under an SM budget once the
+# items outgrow one wave of the register kernel (which has no asynchronous
+# copies to wait for): T = 200 on 148 SMs, about two items per CTA;
+# T = 3000 on 4 SMs, CTAs walking many items each
+@pytest.mark.parametrize("T,num_sms", [(200, 148), (3000, 4)])
+def test_combine_wait_times_out_then_recovers(T, num_sms):
     cfg, b, L, ref = _setup("decode", 31, T, 7168)
     y = b.x.cuda()[torch.from_numpy(np.maximum(ref["recv_src"], 0)).long().cuda()]
     w = b.w.cuda()
-    call = lambda e: ep.ep_combine(y, L.slot_pos, w, d_err=e)  # noqa: E731
+    call = lambda e: ep.ep_combine(y, L.slot_pos, w, num_sms=num_sms, d_err=e)  # noqa: E731
     assert _expired(call) == ep.EP_ERR_TIMEOUT
     out = _normal(call)
     want = oracle.combine(y.cpu(), ref["slot_pos"], b.w)
