@@ -26,8 +26,10 @@
 //    vector of the output.
 //  * combine_reg_kernel (any k <= 32): a warp per item with 128-bit loads
 //    of 8 slot rows at a time into registers.
-//  * combine_fp8_bulk_kernel / combine_fp8_reg_kernel: the same for expert
-//    outputs kept as e4m3 codes plus block scales (below).
+//  * combine_fp8_item_kernel / combine_fp8_bulk_kernel /
+//    combine_fp8_reg_kernel: the same for expert outputs kept as e4m3
+//    codes plus block scales (below); the item kernel on all SMs (k <= 8),
+//    the bulk-copy pipeline under an SM budget (k <= 8, H % 512 == 0).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -385,6 +387,48 @@ __global__ void __launch_bounds__(kQChunkVec)
   }
 }
 
+// k <= 8 and H % 128 == 0, one CTA of kSmallChunkVec threads per (token,
+// chunk of kSmallChunkVec code vectors = 1024 channels), as
+// combine_item_kernel: every thread reads the token's slot rows and
+// weights, then its 16 codes and their block scale of each of the k rows
+// straight into registers, and writes 16 channels of the output.
+__global__ void __launch_bounds__(kSmallChunkVec)
+    combine_fp8_item_kernel(const uint4 *__restrict__ y_q, const float *__restrict__ y_scale,
+                            int T, int H, int k, const int32_t *__restrict__ slot_pos,
+                            const float *__restrict__ w, uint4 *__restrict__ out,
+                            long n_rows) {
+  const int Hq = H >> 4, nb = H >> 7;
+  const int nchunks = (Hq + kSmallChunkVec - 1) / kSmallChunkVec;
+  const int t = blockIdx.x / nchunks;
+  const int v = (blockIdx.x - t * nchunks) * kSmallChunkVec + threadIdx.x;
+  pdl_wait();
+  const long tk = static_cast<long>(t) * k;
+  int row[kBulkMaxK];
+  float wj[kBulkMaxK];
+#pragma unroll
+  for (int j = 0; j < kBulkMaxK; ++j) {
+    const int r = j < k ? __ldg(slot_pos + tk + j) : -1;
+    row[j] = r >= 0 && r < n_rows ? r : -1;  // dropped or out of range: nothing
+    wj[j] = j < k ? (w != nullptr ? __ldg(w + tk + j) : 1.0f) : 0.0f;
+  }
+  if (v >= Hq) return;
+  uint4 q[kBulkMaxK];
+  float sc[kBulkMaxK];
+#pragma unroll
+  for (int j = 0; j < kBulkMaxK; ++j) {
+    q[j] = row[j] >= 0 ? ld_stream_v4(y_q + static_cast<long>(row[j]) * Hq + v)
+                       : make_uint4(0, 0, 0, 0);
+    sc[j] = row[j] >= 0 ? __ldg(y_scale + static_cast<long>(row[j]) * nb + (v >> 3)) : 0.0f;
+  }
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kBulkMaxK; ++j)
+    if (row[j] >= 0) fma_e4m3x16(acc, wj[j], q[j], sc[j]);
+  store_bf16x16(out + (static_cast<long>(t) * Hq + v) * 2, acc);
+}
+
 // Any k <= 32 and H % 128 == 0: a warp per (token, 512 channels), the
 // lane's 16 codes and their scale read directly.
 __global__ void __launch_bounds__(kRegThreads, 2)
@@ -426,6 +470,17 @@ cudaError_t launch_combine_fp8(const void *y_q, const float *y_scale, long n_row
                                void *out, int num_sms, int32_t *d_err, cudaStream_t s,
                                int *launches) {
   const int Hq = H / 16;
+  if (k <= kBulkMaxK && num_sms <= 0) {
+    // all SMs: one CTA per item (waves of CTAs follow one another)
+    const long items = static_cast<long>(T) * ((Hq + kSmallChunkVec - 1) / kSmallChunkVec);
+    if (items == 0) return cudaSuccess;
+    if (items <= kMaxGridX) {
+      ++*launches;
+      return launch_pdl(combine_fp8_item_kernel, dim3(items), dim3(kSmallChunkVec), 0, s, 1,
+                        static_cast<const uint4 *>(y_q), y_scale, T, H, k, slot_pos, w,
+                        static_cast<uint4 *>(out), n_rows);
+    }
+  }
   if (k <= kBulkMaxK && H % 512 == 0 && reinterpret_cast<uintptr_t>(y_scale) % 16 == 0) {
     const long items = static_cast<long>(T) * ((Hq + kQChunkVec - 1) / kQChunkVec);
     if (items == 0) return cudaSuccess;

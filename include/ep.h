@@ -241,8 +241,9 @@ ep_status_t ep_combine(const void *y, int y_rows, int T, int H, int k,
  *   v = fp32_rn(e4m3(y_q[p, c]) * y_scale[p, c / 128])
  *   acc = fma(w[t,j], v, acc) in slot order from 0.0f; out = bf16_rne(acc)
  * y_q       [y_rows, H] e4m3 bytes (16-byte aligned).
- * y_scale   [y_rows, H/128] fp32 (4-byte aligned; 16-byte aligned rows and
- *           H % 512 == 0 take the bulk-copy kernel).
+ * y_scale   [y_rows, H/128] fp32 (4-byte aligned; under an SM budget,
+ *           16-byte aligned rows and H % 512 == 0 take the bulk-copy
+ *           kernel).
  * y_rows, slot_pos, w, out, num_sms, d_err: as ep_combine.  H % 128 == 0.
  */
 ep_status_t ep_combine_fp8(const void *y_q, const float *y_scale, int y_rows,

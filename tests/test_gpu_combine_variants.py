@@ -148,11 +148,12 @@ def test_combine_fp8_decode_full_size():
     _combine_fp8_check(128, 7168, 8, 1)
 
 
+@pytest.mark.parametrize("num_sms", [0, 9])
 @pytest.mark.parametrize("H", [128, 384, 512, 1536, 4096, 7296, 16384])
-def test_combine_fp8_ragged_hidden_and_drops(H):
-    # H % 512 == 0 takes the bulk-copy kernel, other multiples of 128 the
-    # register kernel
-    _combine_fp8_check(97, H, 8, H, drop=0.1)
+def test_combine_fp8_ragged_hidden_and_drops(H, num_sms):
+    # all SMs: the item kernel at every H; under an SM budget H % 512 == 0
+    # takes the bulk-copy kernel, other multiples of 128 the register kernel
+    _combine_fp8_check(97, H, 8, H, drop=0.1, num_sms=num_sms)
 
 
 @pytest.mark.parametrize("k", [1, 3, 16, 32])
@@ -162,7 +163,8 @@ def test_combine_fp8_k(k):
 
 def test_combine_fp8_unit_weights_extra_rows_misaligned_scales():
     _combine_fp8_check(200, 2048, 8, 5, w_none=True, extra_rows=300)
-    _combine_fp8_check(200, 2048, 8, 6, scale_offset=1)     # register kernel
+    _combine_fp8_check(200, 2048, 8, 6, scale_offset=1)     # item kernel
+    _combine_fp8_check(200, 2048, 8, 6, scale_offset=1, num_sms=9)  # register kernel
 
 
 @pytest.mark.parametrize("num_sms", [1, 9])

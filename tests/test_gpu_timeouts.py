@@ -73,11 +73,12 @@ def test_combine_wait_times_out_then_recovers(T, num_sms):
 
 
 def test_combine_fp8_wait_times_out_then_recovers():
+    # the bulk-copy pipeline of the FP8 combine runs under an SM budget
     cfg, b, L, ref = _setup("decode", 32, 300, 7168)
     T, H, k = b.T, b.H, cfg.k
     q, s = ep.ep_dispatch(b.x.cuda(), L.slot_pos, fp8=True)
     w = b.w.cuda()
-    call = lambda e: ep.ep_combine_fp8(q, s, L.slot_pos, w, d_err=e)  # noqa: E731
+    call = lambda e: ep.ep_combine_fp8(q, s, L.slot_pos, w, num_sms=148, d_err=e)  # noqa: E731
     assert _expired(call) == ep.EP_ERR_TIMEOUT
     out = _normal(call)
     want = oracle.combine_fp8(tensor_bytes(q), s.cpu().numpy(), ref["slot_pos"], b.w)
