@@ -271,11 +271,40 @@ __device__ __forceinline__ void decode_e4m3x16(uint4 v, float *f) {
   }
 }
 
+// Packed pairs of fp32 values (sm_100 f32x2 instructions): each lane of
+// fma.rn.f32x2 / mul.rn.f32x2 rounds exactly as the scalar fma.rn.f32 /
+// mul.rn.f32 does, so the chains below are the scalar ones, two at a time
+// (the FP8 combine is issue-bound: 52.6 -> 48.4 us alone at the prefill
+// shape, outputs identical).
+__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(a), "f"(b));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long d, float *a, float *b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(*a), "=f"(*b) : "l"(d));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ void fma_e4m3x16(float *acc, float w, uint4 q, float scale) {
   float f[16];
   decode_e4m3x16(q, f);
+  const unsigned long long w2 = f2_pack(w, w), s2 = f2_pack(scale, scale);
 #pragma unroll
-  for (int e = 0; e < 16; ++e) acc[e] = __fmaf_rn(w, __fmul_rn(f[e], scale), acc[e]);
+  for (int e = 0; e < 16; e += 2) {
+    const unsigned long long a = f2_fma(w2, f2_mul(f2_pack(f[e], f[e + 1]), s2),
+                                        f2_pack(acc[e], acc[e + 1]));
+    f2_unpack(a, &acc[e], &acc[e + 1]);
+  }
 }
 
 __device__ __forceinline__ void store_bf16x16(uint4 *dst, const float *acc) {

@@ -15,7 +15,12 @@ namespace {
 constexpr int kThreads = 256;  // register kernel
 
 constexpr int kFp8BulkThreads = 256;
-constexpr int kFp8InStages = 2;   // bf16 rows in flight per CTA
+// bf16 rows in flight per CTA: two on a persistent grid (a CTA walking a
+// token range loads the next row while it casts this one), one when every
+// token has a CTA of its own (8 CTAs per SM instead of 6: 54.2-55.3 ->
+// 53.3-54.2 us inside the prefill step)
+constexpr int kFp8InStagesRange = 2;
+constexpr int kFp8InStagesOne = 1;
 // Cast rows whose bulk stores may still be reading them.  Two measured
 // slower at the prefill shape (59.5 vs 57.5 us alone): the extra stage
 // costs a CTA per SM (5 instead of 6), which hurts more than the overlap
@@ -32,9 +37,11 @@ constexpr int kFp8OutStages = 1;
 // HBM better than per-lane stores (measured at the prefill shape: 55 us
 // against 57 us for 16-byte stores per lane, 59 us for 512-byte bulk
 // stores per warp, and 61 us for half-row items).
-// 6 CTAs of 256 threads fit an SM's shared memory at H = 7168; the bound
-// keeps registers at or below 42 so that they fit too.
-__global__ void __launch_bounds__(kFp8BulkThreads, 6)
+// At H = 7168, 6 CTAs of 256 threads with two input stages fit an SM's
+// shared memory, 8 with one; the bound keeps registers low enough that
+// they fit too.
+template <int kFp8InStages>
+__global__ void __launch_bounds__(kFp8BulkThreads, kFp8InStages == 1 ? 8 : 6)
     dispatch_fp8_bulk_kernel(const uint4 *__restrict__ x, int T, int H, int k,
                              const int32_t *__restrict__ slot_pos, uint8_t *__restrict__ recv_q,
                              float *__restrict__ recv_scale, long n_rows, int first_polls,
@@ -201,7 +208,9 @@ __global__ void __launch_bounds__(kThreads)
 // Largest hidden size the bulk FP8 kernel stages in shared memory.
 constexpr int kFp8BulkMaxH = 16384;
 
-int fp8_bulk_smem(int H) { return kFp8InStages * 2 * H + kFp8OutStages * (H + H / 32); }
+int fp8_bulk_smem(int in_stages, int H) {
+  return in_stages * 2 * H + kFp8OutStages * (H + H / 32);
+}
 
 cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
                                 const int32_t *slot_pos, void *recv_q,
@@ -211,26 +220,28 @@ cudaError_t launch_dispatch_fp8(const void *x, int T, int H, int k,
   // aligned recv_scale
   if (H % 512 == 0 && H <= kFp8BulkMaxH && reinterpret_cast<uintptr_t>(recv_scale) % 16 == 0) {
     if (T == 0) return cudaSuccess;
-    const int smem = fp8_bulk_smem(H);
-    const cudaError_t err =
-        raise_dynamic_smem(reinterpret_cast<const void *>(dispatch_fp8_bulk_kernel),
-                           fp8_bulk_smem(kFp8BulkMaxH));
-    if (err != cudaSuccess) return err;
     // all SMs: one token per CTA, waves of CTAs following one another as
     // SMs free up (measured against a persistent grid of 6 CTAs per SM:
     // 57.5-62 -> 54.2-55.3 us inside the prefill step, 49-52 -> 46-47 us
     // alone); under an SM budget a persistent grid sized to it
-    const long grid =
-        num_sms > 0
-            ? persistent_grid(reinterpret_cast<const void *>(dispatch_fp8_bulk_kernel),
-                              kFp8BulkThreads, smem,
-                              static_cast<long>(T) * (kFp8BulkThreads / kWarp), num_sms)
-            : static_cast<long>(T);
-    ++*launches;
-    return launch_pdl(dispatch_fp8_bulk_kernel, dim3(grid), dim3(kFp8BulkThreads), smem, s, 1,
-                      static_cast<const uint4 *>(x), T, H, k, slot_pos,
-                      static_cast<uint8_t *>(recv_q), recv_scale, n_rows, first_wait_polls(),
-                      d_err);
+    auto launch = [&](auto kern, int in_stages, long grid) -> cudaError_t {
+      const cudaError_t err = raise_dynamic_smem(reinterpret_cast<const void *>(kern),
+                                                 fp8_bulk_smem(in_stages, kFp8BulkMaxH));
+      if (err != cudaSuccess) return err;
+      ++*launches;
+      return launch_pdl(kern, dim3(grid), dim3(kFp8BulkThreads), fp8_bulk_smem(in_stages, H), s,
+                        1, static_cast<const uint4 *>(x), T, H, k, slot_pos,
+                        static_cast<uint8_t *>(recv_q), recv_scale, n_rows, first_wait_polls(),
+                        d_err);
+    };
+    if (num_sms <= 0)
+      return launch(dispatch_fp8_bulk_kernel<kFp8InStagesOne>, kFp8InStagesOne,
+                    static_cast<long>(T));
+    auto kern = dispatch_fp8_bulk_kernel<kFp8InStagesRange>;
+    const long grid = persistent_grid(reinterpret_cast<const void *>(kern), kFp8BulkThreads,
+                                      fp8_bulk_smem(kFp8InStagesRange, H),
+                                      static_cast<long>(T) * (kFp8BulkThreads / kWarp), num_sms);
+    return launch(kern, kFp8InStagesRange, grid);
   }
   const long nchunks = (H / 128 + 3) / 4;
   const long items = static_cast<long>(T) * nchunks;
