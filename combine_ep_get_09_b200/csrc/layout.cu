@@ -98,7 +98,13 @@ __device__ __forceinline__ long long raw_id(const IdT *idx, long i, int /*k*/) {
 }
 template <>
 __device__ __forceinline__ long long raw_id<uint8_t>(const uint8_t *idx, long i, int k) {
-  return idx[i] ? static_cast<long long>(i % k) : -1;
+  return idx[i] ? static_cast<long long>(static_cast<unsigned>(i) % static_cast<unsigned>(k)) : -1;
+}
+
+// Token of flat slot i: slots number fewer than 2^31, so the 32-bit
+// unsigned division is exact and far cheaper than a 64-bit one.
+__device__ __forceinline__ int32_t token_of_slot(long i, int k) {
+  return static_cast<int32_t>(static_cast<unsigned>(i) / static_cast<unsigned>(k));
 }
 
 // Ids are read kIdBatch at a time per lane, all loads issued before any is
@@ -280,7 +286,7 @@ __device__ void place_segment(const IdT *idx, long beg, long end, int k, int E,
       const int q = sr.packed[b];
       const int pos = q >= 0 ? warp_base(q & 1023, base_w, add1, add2) + (q >> 10) : -1;
       slot_pos[i] = pos;
-      if (pos >= 0) recv_src[pos] = static_cast<int32_t>(i / k);
+      if (pos >= 0) recv_src[pos] = token_of_slot(i, k);
     }
   }
   for (long c0 = beg + 32 * kRegChunks; c0 < end; c0 += 32 * kIdBatch) {
@@ -293,7 +299,7 @@ __device__ void place_segment(const IdT *idx, long beg, long end, int k, int E,
         const int e = check_id(v[b], E, nullptr);
         const int pos = e >= 0 ? warp_base(e, base_w, add1, add2) + slot_pos[i] : -1;
         slot_pos[i] = pos;
-        if (pos >= 0) recv_src[pos] = static_cast<int32_t>(i / k);
+        if (pos >= 0) recv_src[pos] = token_of_slot(i, k);
       }
     }
   }

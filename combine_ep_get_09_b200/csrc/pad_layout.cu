@@ -88,7 +88,8 @@ __global__ void __launch_bounds__(kPadThreads)
     if (row >= 0 && row < kept) {
       const int e = segment_of(off, E, row);
       out = offp[e] + (row - off[e]);
-      recv_src_pad[out] = static_cast<int32_t>(i / k);
+      // slots number fewer than 2^31: an exact 32-bit division
+      recv_src_pad[out] = static_cast<int32_t>(static_cast<unsigned>(i) / static_cast<unsigned>(k));
     }
     slot_pos_pad[i] = out;
   }
