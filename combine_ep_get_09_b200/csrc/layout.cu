@@ -224,6 +224,32 @@ __device__ __forceinline__ int rank_one(int e, int bits, int *hist_w) {
   return r;
 }
 
+// Slots past the register chunks (CTA shares above 32 * kRegChunks slots
+// a warp), out of line: code a launch does not run stays out of the way of
+// the code it does, which the SMs fetch cold after the caches are flushed
+// (prefill layout 13.2 -> 9.5 us a launch after a flush, 8.8 -> 8.6 warm).
+template <typename IdT>
+__device__ __noinline__ void rank_rest(const IdT *idx, long from, long end, int k, int E, int bits,
+                                       int32_t *d_err, int *hist_w, int32_t *slot_pos,
+                                       short *ids_smem, long cta_beg) {
+  const int lane = threadIdx.x & 31;
+  for (long c0 = from; c0 < end; c0 += 32 * kIdBatch) {
+    long long v[kIdBatch];
+    load_id_batch(idx, c0, end, k, v);
+#pragma unroll
+    for (int b = 0; b < kIdBatch; ++b) {
+      if (c0 + 32 * b >= end) break;  // uniform across the warp
+      const long i = c0 + 32 * b + lane;
+      const int e = check_id(v[b], E, d_err);
+      const int r = rank_one(e, bits, hist_w);
+      if (i < end) {
+        slot_pos[i] = r;
+        if (ids_smem != nullptr) ids_smem[i - cta_beg] = static_cast<short>(e);
+      }
+    }
+  }
+}
+
 // ids_smem (optional): the checked ids of the CTA's slots, indexed from
 // cta_beg, for the token-mask pass to read from shared memory.
 template <typename IdT>
@@ -247,21 +273,9 @@ __device__ void rank_segment(const IdT *idx, long beg, long end, const Params &p
       }
     }
   }
-  for (long c0 = beg + 32 * kRegChunks; c0 < end; c0 += 32 * kIdBatch) {
-    long long v[kIdBatch];
-    load_id_batch(idx, c0, end, p.k, v);
-#pragma unroll
-    for (int b = 0; b < kIdBatch; ++b) {
-      if (c0 + 32 * b >= end) break;  // uniform across the warp
-      const long i = c0 + 32 * b + lane;
-      const int e = check_id(v[b], E, d_err);
-      const int r = rank_one(e, bits, hist_w);
-      if (i < end) {
-        slot_pos[i] = r;
-        if (ids_smem != nullptr) ids_smem[i - cta_beg] = static_cast<short>(e);
-      }
-    }
-  }
+  if (beg + 32 * kRegChunks < end)
+    rank_rest(idx, beg + 32 * kRegChunks, end, p.k, E, bits, d_err, hist_w, slot_pos, ids_smem,
+              cta_beg);
 }
 
 // The first row of expert e for this warp: base_w[e] (+ add1[e] + add2[e]
@@ -271,6 +285,28 @@ __device__ __forceinline__ int warp_base(int e, const int *base_w, const int *ad
   int b = base_w[e];
   if (add1 != nullptr) b += add1[e] + add2[e];
   return b;
+}
+
+// place_segment's counterpart of rank_rest, out of line for the same reason.
+template <typename IdT>
+__device__ __noinline__ void place_rest(const IdT *idx, long from, long end, int k, int E,
+                                        const int *base_w, int32_t *slot_pos, int32_t *recv_src,
+                                        const int *add1, const int *add2) {
+  const int lane = threadIdx.x & 31;
+  for (long c0 = from; c0 < end; c0 += 32 * kIdBatch) {
+    long long v[kIdBatch];
+    load_id_batch(idx, c0, end, k, v);
+#pragma unroll
+    for (int b = 0; b < kIdBatch; ++b) {
+      const long i = c0 + 32 * b + lane;
+      if (i < end) {
+        const int e = check_id(v[b], E, nullptr);
+        const int pos = e >= 0 ? warp_base(e, base_w, add1, add2) + slot_pos[i] : -1;
+        slot_pos[i] = pos;
+        if (pos >= 0) recv_src[pos] = token_of_slot(i, k);
+      }
+    }
+  }
 }
 
 template <typename IdT>
@@ -289,20 +325,29 @@ __device__ void place_segment(const IdT *idx, long beg, long end, int k, int E,
       if (pos >= 0) recv_src[pos] = token_of_slot(i, k);
     }
   }
-  for (long c0 = beg + 32 * kRegChunks; c0 < end; c0 += 32 * kIdBatch) {
+  if (beg + 32 * kRegChunks < end)
+    place_rest(idx, beg + 32 * kRegChunks, end, k, E, base_w, slot_pos, recv_src, add1, add2);
+}
+
+// Bit r set when token t has a kept slot in rank r, from the ids in
+// global memory (the CTAs whose ids are not staged in shared memory), out
+// of line as rank_rest is.
+template <typename IdT>
+__device__ __noinline__ unsigned long long token_rank_bits(const IdT *idx, int t, int k, int E,
+                                                           unsigned long long g_magic) {
+  const long base = static_cast<long>(t) * k;
+  unsigned long long m = 0;
+  for (int j0 = 0; j0 < k; j0 += kIdBatch) {
     long long v[kIdBatch];
-    load_id_batch(idx, c0, end, k, v);
+#pragma unroll
+    for (int b = 0; b < kIdBatch; ++b) v[b] = j0 + b < k ? raw_id(idx, base + j0 + b, k) : -1;
 #pragma unroll
     for (int b = 0; b < kIdBatch; ++b) {
-      const long i = c0 + 32 * b + lane;
-      if (i < end) {
-        const int e = check_id(v[b], E, nullptr);
-        const int pos = e >= 0 ? warp_base(e, base_w, add1, add2) + slot_pos[i] : -1;
-        slot_pos[i] = pos;
-        if (pos >= 0) recv_src[pos] = token_of_slot(i, k);
-      }
+      const int e = check_id(v[b], E, nullptr);
+      if (e >= 0) m |= 1ull << ((static_cast<unsigned long long>(e) * g_magic) >> 32);
     }
   }
+  return m;
 }
 
 // Token-in-rank mask rows for tokens [t_beg, t_end).  Per-rank token counts
@@ -324,18 +369,7 @@ __device__ void rank_mask(const Params &p, int t_beg, int t_end, int *hist_w,
         if (e >= 0) m |= 1ull << rank_of(e, p);
       }
     } else if (t < t_end) {
-      const long base = static_cast<long>(t) * p.k;
-      for (int j0 = 0; j0 < p.k; j0 += kIdBatch) {
-        long long v[kIdBatch];
-#pragma unroll
-        for (int b = 0; b < kIdBatch; ++b)
-          v[b] = j0 + b < p.k ? raw_id(idx, base + j0 + b, p.k) : -1;
-#pragma unroll
-        for (int b = 0; b < kIdBatch; ++b) {
-          const int e = check_id(v[b], p.E, nullptr);
-          if (e >= 0) m |= 1ull << rank_of(e, p);
-        }
-      }
+      m = token_rank_bits(idx, t, p.k, p.E, p.g_magic);
     }
     if (t < t_end && p.in_rank != nullptr) {
       uint8_t *row = p.in_rank + static_cast<long>(t) * p.R;
