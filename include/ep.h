@@ -165,7 +165,11 @@ ep_status_t ep_get_layout(const void *idx, int idx_is_int64, int T, int k,
  *             ep_aligned_rows(T, k, E, align).
  * T >= 0, 1 <= k <= EP_MAX_K, H > 0 with H % 8 == 0 (H % 128 == 0 for
  * fp8), T*k < 2^31.
- * num_sms     SMs to spread the work over (0 = all of them).
+ * num_sms     SMs to spread the work over.  0 = all of them: one CTA (or
+ *             warp) per work item, waves of CTAs following one another as
+ *             SMs free up.  n > 0: a persistent grid of the CTAs that n SMs
+ *             hold at once, so that kernels on other streams keep the
+ *             other SMs (the CTAs are not pinned to particular SMs).
  * d_err       optional device error word (see the conventions above).
  */
 ep_status_t ep_dispatch(const void *x, int T, int H, int k,
