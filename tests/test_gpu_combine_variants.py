@@ -192,6 +192,30 @@ def test_combine_fp8_special_codes():
     np.testing.assert_array_equal(tensor_bits16(out), oracle.combine_fp8(q, s, slot, w))
 
 
+@pytest.mark.parametrize("num_sms", [0, 9])
+def test_combine_fp8_subnormal_products(num_sms):
+    # scales at and below the fp32 normal range, so that scaled values and
+    # the fma chain run through fp32 subnormals: the packed f32x2 multiply
+    # and fma must keep them exactly as the oracle's scalar fp32 does
+    rng = np.random.default_rng(77)
+    T, k, H = 64, 4, 1024
+    n = T * k
+    q = rng.integers(0, 256, size=(n, H), dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x01  # no NaN codes
+    choices = np.array([1.1754944e-38, 1e-38, 1e-40, 2.0 ** -140, 1.4e-45, 3e-42],
+                       np.float32)
+    s = rng.choice(choices, size=(n, H // 128)).astype(np.float32)
+    slot = rng.permutation(n).astype(np.int32).reshape(T, k)
+    w = rng.random((T, k)).astype(np.float32)
+    w[:, 0] = 1.0
+    out = ep.ep_combine_fp8(torch.from_numpy(q).cuda().view(torch.float8_e4m3fn),
+                            torch.from_numpy(s).cuda(), torch.from_numpy(slot).cuda(),
+                            torch.from_numpy(w).cuda(), num_sms=num_sms)
+    want = oracle.combine_fp8(q, s, slot, w)
+    assert (want & 0x7F80 == 0).any()  # some outputs are bf16 subnormals
+    np.testing.assert_array_equal(tensor_bits16(out), want)
+
+
 # -------------------------------------------------------------- replicas
 
 def _replica_table(rng, E, hot, copies):

@@ -328,6 +328,26 @@ def test_combine_sm_budget(T, num_sms):
     assert _combine_check(cfg, b, num_sms=num_sms) == 1.0
 
 
+@pytest.mark.parametrize("num_sms", [0, 9])
+def test_combine_subnormal_values(num_sms):
+    # expert outputs that are bf16 subnormals and tiny normals, weights
+    # below 1: the fp32 chain and the final bf16 rounding run through
+    # subnormals and must match the oracle bit for bit
+    rng = np.random.default_rng(78)
+    T, k, H = 96, 8, 1024
+    n = T * k
+    mag = rng.integers(1, 0x0100, size=(n, H)).astype(np.uint16)   # exponent 0 or 1
+    sign = (rng.random((n, H)) < 0.5).astype(np.uint16) << 15
+    y = torch.from_numpy((mag | sign).view(np.int16)).view(torch.bfloat16)
+    slot = rng.permutation(n).astype(np.int32).reshape(T, k)
+    w = (rng.random((T, k)) * 0.9).astype(np.float32)
+    out = ep.ep_combine(y.cuda(), torch.from_numpy(slot).cuda(), torch.from_numpy(w).cuda(),
+                        num_sms=num_sms)
+    want = oracle.combine(y, slot, torch.from_numpy(w))
+    assert (want & 0x7F80 == 0).any()
+    np.testing.assert_array_equal(tensor_bits16(out), want)
+
+
 def test_combine_k32_and_k1():
     for k, E in ((32, 64), (1, 4)):
         cfg = workloads.Config("k", 200, 512, E, 4, k, "uniform", ("bf16",), "scale")
