@@ -85,14 +85,17 @@ def test_combine_fp8_wait_times_out_then_recovers():
     np.testing.assert_array_equal(tensor_bits16(out), want)
 
 
-def test_dispatch_fp8_wait_times_out_then_recovers():
+# all SMs: one token per CTA (a single wait each); under an SM budget:
+# CTAs walking token ranges with two rows in flight
+@pytest.mark.parametrize("num_sms", [0, 7])
+def test_dispatch_fp8_wait_times_out_then_recovers(num_sms):
     cfg, b, L, ref = _setup("prefill", 33, 1000, 7168)
     T, H, k = b.T, b.H, cfg.k
     x = b.x.cuda()
     q = torch.empty((T * k, H), dtype=torch.float8_e4m3fn, device="cuda")
     s = torch.empty((T * k, H // 128), dtype=torch.float32, device="cuda")
     call = lambda e: ep.ep_dispatch(x, L.slot_pos, fp8=True, recv=q,  # noqa: E731
-                                    recv_scale=s, d_err=e)
+                                    recv_scale=s, num_sms=num_sms, d_err=e)
     assert _expired(call) == ep.EP_ERR_TIMEOUT
     _normal(call)
     wq, ws_ = oracle.dispatch_fp8(b.x, ref["slot_pos"], T * k)
