@@ -34,3 +34,40 @@ def test_cpu_baseline_reports_both_legs():
     allc = res["all_cores"]
     assert allc["kind"] == "oracle" and allc["cores"] >= 1 and allc["value"] > 0
     assert "threads" in allc["sample"]
+
+
+def test_profiled_traffic_only_while_the_sources_match(tmp_path, monkeypatch):
+    # the roofline's traffic figure is read back only for the code it was
+    # captured on: a recorded digest that differs from the current sources'
+    # (or a missing entry, or no file) gives None
+    import json
+    f = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.profiled_traffic("combine") is None
+    rec = {"combine": {"traffic_bytes_per_launch": 123456,
+                       "source_sha256": bench.kernel_source_digest("combine")},
+           "dispatch_bf16": {"traffic_bytes_per_launch": 7,
+                             "source_sha256": "0" * 64}}
+    f.write_text(json.dumps(rec))
+    assert bench.profiled_traffic("combine") == 123456.0
+    assert bench.profiled_traffic("dispatch_bf16") is None
+    assert bench.profiled_traffic("layout") is None
+
+
+def test_kernel_digests_cover_distinct_sources():
+    # every kernel named in the roofline has a digest over its own files;
+    # kernels built from the same files share one
+    d = {k: bench.kernel_source_digest(k) for k in bench.KERNEL_SOURCES}
+    assert all(len(v) == 64 for v in d.values())
+    assert d["combine"] == d["combine_fp8"]
+    assert len({d["layout"], d["dispatch_bf16"], d["dispatch_fp8"], d["combine"]}) == 4
+
+
+def test_workload_config_names_the_step_and_its_bytes():
+    cfg = workloads.CONFIGS["prefill"]
+    c = bench.workload_config(cfg, 1)
+    assert c["workload"].startswith("prefill")
+    assert (c["T"], c["H"], c["E"], c["R"], c["k"]) == (4096, 7168, 256, 8, 8)
+    assert c["bytes_per_step"] == sum(bench.step_bytes(4096, 7168, 8, 256, 8).values())
+    assert "flushed" in c["l2"]
+    assert "model" not in c
