@@ -41,8 +41,9 @@ namespace cg = cooperative_groups;
 // CTA sizes of the cluster kernel: 512 threads while a CTA's slots fit the
 // warps' registers (at most 4096 slots: 8 chunks of 32 per warp), which
 // leaves room for 128 registers a thread; 1024 above that (64 registers).
-// Measured at the prefill shape (2048 slots a CTA): 512 threads 13.3-13.8
-// us per launch after an L2 flush, 1024 threads 15.0 us.
+// Measured at the prefill shape (2048 slots a CTA, 16 CTAs): 512 threads
+// 9.2-9.5 us per launch after an L2 flush, 256 threads 10.5, 1024 threads
+// 11.8-12.0; 3072 or 4096 slots a CTA (11 or 8 CTAs) 9.9-11.2 us.
 constexpr int kClusterThreads = 1024;
 constexpr int kClusterThreadsSmall = 512;
 constexpr long kClusterSmallCtaSlots = 4096;
